@@ -1,0 +1,333 @@
+"""IQ8R oracle -- TEST INFRASTRUCTURE ONLY.
+
+A plain, slow, CPU restatement of the IQ8R rotated W8A8 linear layer, written
+to check the CUDA library against. Only the tests, the package's ``smoke()``
+and the CPU-baseline leg of ``bench.py`` may import it; the library never
+does, and the two share no code.
+
+What it follows (the pages are model cards of the "radiance" engine):
+
+* "Qwen3.8-27B IQ8R + DFlash2 -- radiance container", table row "Weights":
+  every trunk linear is int8 with codes -127..127, a u8 scale per row and
+  256 of K under a bf16 scale per row, each 128 of K rotated by the
+  unnormalised Hadamard; the lm_head is int8 with a bf16 scale per row and
+  128 of K.
+* same page, table row "Activations": int8 under the same rotation (W8A8).
+* same page, "How this file was made", the recipe rules
+  ``codes=i8 group=256 scale=u8 scale2=bf16 block2=1x* transform=fwht128
+  clamp=sym`` (trunk) and ``codes=i8 group=128 scale=bf16 clamp=sym``
+  (lm_head).
+* "Qwen3.8-Flash-Next, IQR-V4 -- radiance container", row "Routed experts":
+  the transform is the 128-point Walsh-Hadamard rotation.
+
+Where the pages are silent the oracle writes down a stated definition (the
+library follows it exactly):
+
+* fp32 transform order: radix-2 butterflies, h = 1, 2, 4, ..., 64, each
+  (a, b) -> (a + b, a - b) with round-to-nearest-even, no fused ops;
+* activation scale: one per token (row), a = amax / 127, codes
+  rint(x' * (127 / amax)) clamped to +-127;
+* trunk scales: step d[n, g] = float(s2[n]) * s1[n, g]; s2 = bf16 of
+  R[n] / (127 * 255) rounded up, s1 = min(255, ceil(A[n, g] / (127 * s2)));
+* lm_head scale: s[n, g] = bf16 of A[n, g] / 127 rounded up;
+* rounding: round-half-to-even wherever a value is rounded to nearest;
+* the factor 1/128 (H H = 128 I) is applied to the output.
+
+Parity unpinned: the choice of the three scale rules above (per-token
+activation scale, the s2/s1 composition, the lm_head scale rule) and of the
+butterfly order. They are stated definitions, not facts the pages fix; the
+tests pin everything that follows from them.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "GROUP_TRUNK",
+    "GROUP_HEAD",
+    "CODE_MAX",
+    "SUB_MAX",
+    "bf16_to_f32",
+    "f32_to_bf16_exact",
+    "bf16_round_up",
+    "bf16_round_nearest",
+    "hadamard128",
+    "fwht128_f32",
+    "fwht128_f64",
+    "act_quant",
+    "pack",
+    "packed_sizes",
+    "partials",
+    "linear",
+    "linear_bf16",
+]
+
+GROUP_TRUNK = 256  # "a u8 scale per row and 256 of K" (IQ8R page, "Weights")
+GROUP_HEAD = 128   # "a bf16 scale per row and 128" (IQ8R page, "Weights")
+CODE_MAX = 127     # "codes -127..127", clamp=sym (IQ8R page, "Weights" and recipe)
+SUB_MAX = 255      # largest u8 sub-scale (recipe: scale=u8)
+ROT = 128          # fwht128: the rotation acts on each 128 of K
+
+
+# ---------------------------------------------------------------- bf16 helpers
+
+def bf16_to_f32(bits: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> float32 values (exact widening)."""
+    b = np.asarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def f32_to_bf16_exact(v: np.ndarray) -> np.ndarray:
+    """float32 values that are already bf16-representable -> bit patterns."""
+    u = np.ascontiguousarray(v, dtype=np.float32).view(np.uint32)
+    if np.any(u & np.uint32(0xFFFF)):
+        raise ValueError("value is not representable in bf16")
+    return (u >> np.uint32(16)).astype(np.uint16)
+
+
+_BF16_MIN_NORMAL = 2.0 ** -126
+_BF16_SUB_EXP = 133  # bf16 subnormal spacing is 2**-133 (7 stored mantissa bits)
+
+
+def bf16_round_up(v: np.ndarray) -> np.ndarray:
+    """Smallest bf16 value >= v, for finite v >= 0. Returns float32 values.
+
+    Written from the format: a normal bf16 carries 8 significant bits, so a
+    value m * 2**e (m in [0.5, 1)) rounds up to ceil(m * 2**8) * 2**(e - 8);
+    below 2**-126 the grid is the subnormal one, multiples of 2**-133.
+    """
+    x = np.asarray(v, dtype=np.float64)
+    if np.any(x < 0) or not np.all(np.isfinite(x)):
+        raise ValueError("bf16_round_up expects finite non-negative input")
+    m, e = np.frexp(x)
+    normal = np.ldexp(np.ceil(np.ldexp(m, 8)), e - 8)
+    sub = np.ldexp(np.ceil(np.ldexp(x, _BF16_SUB_EXP)), -_BF16_SUB_EXP)
+    r = np.where(x >= _BF16_MIN_NORMAL, normal, sub)
+    with np.errstate(over="ignore"):
+        return r.astype(np.float32)
+
+
+def bf16_round_nearest(v: np.ndarray) -> np.ndarray:
+    """Round float64 values to bf16, nearest with ties to even; bit patterns.
+
+    Same grid as ``bf16_round_up``; ``np.rint`` rounds halves to even.
+    Values past the largest bf16 (and its half-ulp) become +-inf.
+    """
+    x = np.asarray(v, dtype=np.float64)
+    m, e = np.frexp(x)
+    normal = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)
+    sub = np.ldexp(np.rint(np.ldexp(x, _BF16_SUB_EXP)), -_BF16_SUB_EXP)
+    r = np.where(np.abs(x) >= _BF16_MIN_NORMAL, normal, sub)
+    with np.errstate(over="ignore"):
+        r32 = r.astype(np.float32)  # exact, or +-inf past the bf16 range
+    return (np.ascontiguousarray(r32).view(np.uint32) >> np.uint32(16)).astype(np.uint16)
+
+
+# ----------------------------------------------------------------- transform
+
+def hadamard128() -> np.ndarray:
+    """The 128x128 unnormalised Hadamard matrix, natural (Sylvester) order.
+
+    H[i][j] = (-1) ** popcount(i & j): the "unnormalised Hadamard" of the
+    IQ8R page ("Weights") and the "128-point Walsh-Hadamard rotation" of the
+    Flash-Next page ("Routed experts"). No 1/sqrt(128) factor.
+    """
+    i = np.arange(ROT)
+    a = i[:, None] & i[None, :]
+    pc = np.zeros_like(a)
+    for bit in range(7):
+        pc += (a >> bit) & 1
+    return np.where(pc % 2 == 0, 1, -1).astype(np.int64)
+
+
+def fwht128_f32(v: np.ndarray) -> np.ndarray:
+    """fwht128 of each consecutive 128 of the last axis, in float32.
+
+    Stated definition of the fp32 arithmetic (the pages give none): radix-2
+    butterflies in place, stage h = 1, 2, 4, ..., 64 in that order; for every
+    index i with (i & h) == 0 the pair (v[i], v[i+h]) becomes
+    (v[i] + v[i+h], v[i] - v[i+h]), each an IEEE float32 add or subtract.
+    Within a stage the butterflies are independent, so doing them together
+    changes no rounding.
+    """
+    v = np.asarray(v, dtype=np.float32)
+    if v.shape[-1] % ROT:
+        raise ValueError("last axis must be a multiple of 128")
+    x = v.reshape(-1, ROT).copy()
+    h = 1
+    while h < ROT:
+        y = x.reshape(x.shape[0], ROT // (2 * h), 2, h)
+        lo = y[:, :, 0, :].copy()
+        hi = y[:, :, 1, :].copy()
+        y[:, :, 0, :] = lo + hi
+        y[:, :, 1, :] = lo - hi
+        h *= 2
+    return x.reshape(v.shape)
+
+
+def fwht128_f64(v: np.ndarray) -> np.ndarray:
+    """fwht128 in float64 as the matrix product with ``hadamard128()``."""
+    v = np.asarray(v, dtype=np.float64)
+    if v.shape[-1] % ROT:
+        raise ValueError("last axis must be a multiple of 128")
+    H = hadamard128().astype(np.float64)
+    return (v.reshape(-1, ROT) @ H.T).reshape(v.shape)
+
+
+# ------------------------------------------------------------ activations
+
+def act_quant(x_bits: np.ndarray, rotate: bool = True):
+    """Rotate and quantise activations to int8, one scale per token.
+
+    "int8 under the same rotation (W8A8)" (IQ8R page, "Activations"). The
+    granularity is not given; the stated definition is per token (row):
+
+      x' = fwht128(x) in float32 (or x itself when ``rotate`` is false),
+      amax = max |x'|, inv = 127 / amax (float32 divide),
+      q = clamp(rint(x' * inv), -127, 127), a = amax / 127 (float32).
+
+    A row with amax == 0 gives a = 0 and all-zero codes.
+    Returns (q int8 [M, K], a float32 [M]).
+    """
+    x = bf16_to_f32(x_bits)
+    if x.ndim != 2:
+        raise ValueError("x must be [M, K]")
+    xr = fwht128_f32(x) if rotate else x.copy()
+    amax = np.max(np.abs(xr), axis=1) if xr.shape[1] else np.zeros(xr.shape[0], np.float32)
+    q = np.zeros(xr.shape, dtype=np.int8)
+    a = np.zeros(xr.shape[0], dtype=np.float32)
+    nz = amax > 0
+    if np.any(nz):
+        inv = np.float32(CODE_MAX) / amax[nz]
+        t = xr[nz] * inv[:, None]
+        q[nz] = np.clip(np.rint(t), -CODE_MAX, CODE_MAX).astype(np.int8)
+        a[nz] = amax[nz] / np.float32(CODE_MAX)
+    return q, a
+
+
+# ---------------------------------------------------------------- weights
+
+def packed_sizes(fmt: str, n: int, k: int):
+    """Byte sizes of (codes, sub-scales, scales) for a packed [n, k] weight."""
+    if fmt == "g256":
+        return n * k, n * (k // GROUP_TRUNK), 2 * n
+    if fmt == "g128":
+        return n * k, 0, 2 * n * (k // GROUP_HEAD)
+    raise ValueError(fmt)
+
+
+def pack(w_bits: np.ndarray, fmt: str = "g256", rotate: bool = True):
+    """Round-to-nearest packing of a bf16 weight [N, K] (the recipe's ``rtn``).
+
+    Trunk, ``fmt="g256"`` (recipe ``codes=i8 group=256 scale=u8 scale2=bf16
+    block2=1x* transform=fwht128 clamp=sym``). Stated composition d = s2*s1:
+
+      W' = fwht128(W) in float32,
+      A[n, g] = max |W'| over the 256-block g,  R[n] = max_g A[n, g],
+      s2[n] = bf16 of float32(R / 32385) rounded up (32385 = 127 * 255),
+      s1[n, g] = min(255, ceil(A / (127 * s2))) (float32 divide), 0 if s2 = 0,
+      codes = clamp(rint(W' / (s2 * s1)), -127, 127) (float32 divide),
+      0 where s2 * s1 = 0.
+
+    lm_head, ``fmt="g128"`` (recipe ``codes=i8 group=128 scale=bf16
+    clamp=sym``): s[n, g] = bf16 of float32(A / 127) rounded up over each
+    128-block; codes = clamp(rint(W' / s), -127, 127), 0 where s = 0.
+
+    Returns (codes int8 [N, K], sub uint8 [N, K/256] or None,
+    scale bf16 bits: [N] for g256, [N, K/128] for g128).
+    """
+    w = bf16_to_f32(w_bits)
+    if w.ndim != 2:
+        raise ValueError("w must be [N, K]")
+    n, k = w.shape
+    wr = fwht128_f32(w) if rotate else w.copy()
+    if fmt == "g256":
+        if k % GROUP_TRUNK:
+            raise ValueError("K must be a multiple of 256")
+        ng = k // GROUP_TRUNK
+        blocks = wr.reshape(n, ng, GROUP_TRUNK)
+        A = np.max(np.abs(blocks), axis=2)                       # float32 [n, ng]
+        R = np.max(A, axis=1)                                   # float32 [n]
+        s2 = bf16_round_up(R / np.float32(CODE_MAX * SUB_MAX))  # float32 [n]
+        den = np.float32(CODE_MAX) * s2                         # exact (8 x 7 bits)
+        s1 = np.zeros((n, ng), dtype=np.float32)
+        ok = s2 > 0
+        if np.any(ok):
+            s1[ok] = np.minimum(np.float32(SUB_MAX), np.ceil(A[ok] / den[ok, None]))
+        d = s2[:, None] * s1                                    # exact (8 x 8 bits)
+        codes = np.zeros((n, ng, GROUP_TRUNK), dtype=np.int8)
+        dz = d > 0
+        if np.any(dz):
+            t = blocks[dz] / d[dz][:, None]
+            codes[dz] = np.clip(np.rint(t), -CODE_MAX, CODE_MAX).astype(np.int8)
+        return codes.reshape(n, k), s1.astype(np.uint8), f32_to_bf16_exact(s2)
+    if fmt == "g128":
+        if k % GROUP_HEAD:
+            raise ValueError("K must be a multiple of 128")
+        ng = k // GROUP_HEAD
+        blocks = wr.reshape(n, ng, GROUP_HEAD)
+        A = np.max(np.abs(blocks), axis=2)
+        s = bf16_round_up(A / np.float32(CODE_MAX))             # float32 [n, ng]
+        codes = np.zeros((n, ng, GROUP_HEAD), dtype=np.int8)
+        sz = s > 0
+        if np.any(sz):
+            t = blocks[sz] / s[sz][:, None]
+            codes[sz] = np.clip(np.rint(t), -CODE_MAX, CODE_MAX).astype(np.int8)
+        return codes.reshape(n, k), None, f32_to_bf16_exact(s)
+    raise ValueError(fmt)
+
+
+# ------------------------------------------------------------------ linear
+
+def partials(xq: np.ndarray, codes: np.ndarray, group: int) -> np.ndarray:
+    """P[m, n, g] = sum over block g of xq[m, k] * codes[n, k], exact int64.
+
+    Each block product is a float64 matrix product of small integers: every
+    term is below 2**14 and every block sum below 2**22 in magnitude, so the
+    float64 result is the exact integer whatever the summation order.
+    """
+    xq = np.asarray(xq)
+    codes = np.asarray(codes)
+    m, k = xq.shape
+    n, k2 = codes.shape
+    if k != k2 or k % group:
+        raise ValueError("shape mismatch")
+    ng = k // group
+    out = np.empty((m, n, ng), dtype=np.int64)
+    for g in range(ng):
+        xs = xq[:, g * group:(g + 1) * group].astype(np.float64)
+        ws = codes[:, g * group:(g + 1) * group].astype(np.float64)
+        out[:, :, g] = np.rint(xs @ ws.T).astype(np.int64)
+    return out
+
+
+def linear(xq: np.ndarray, a: np.ndarray, fmt: str, codes: np.ndarray,
+           sub: np.ndarray | None, scale_bits: np.ndarray, rotated: bool = True) -> np.ndarray:
+    """The layer output in float64 before its bf16 rounding, y64 [M, N].
+
+    Trunk: y = a[m] * s2[n] * S[m, n] / 128, S = sum_g s1[n, g] * P[m, n, g]
+    (S exact in int64). lm_head: y = a[m] / 128 * sum_g s[n, g] * P[m, n, g]
+    (each term and the sum exact in float64). The 1/128 undoes H H = 128 I
+    and is dropped when the weight was packed unrotated.
+    """
+    a64 = np.asarray(a, dtype=np.float32).astype(np.float64)
+    if fmt == "g256":
+        P = partials(xq, codes, GROUP_TRUNK)
+        S = np.einsum("mng,ng->mn", P, np.asarray(sub).astype(np.int64))
+        s2 = bf16_to_f32(scale_bits).astype(np.float64)
+        y = a64[:, None] * s2[None, :] * S.astype(np.float64)
+    elif fmt == "g128":
+        P = partials(xq, codes, GROUP_HEAD)
+        s = bf16_to_f32(scale_bits).astype(np.float64)
+        y = a64[:, None] * np.einsum("mng,ng->mn", P.astype(np.float64), s)
+    else:
+        raise ValueError(fmt)
+    if rotated:
+        y = y / 128.0
+    return y
+
+
+def linear_bf16(y64: np.ndarray) -> np.ndarray:
+    """bf16 output bits: y64 rounded to nearest, ties to even."""
+    return bf16_round_nearest(y64)

@@ -1,0 +1,167 @@
+"""The oracle against what the pages and the mathematics fix (CPU only)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import pins
+from iq8r_inputs import WORKLOADS, gen_workload
+
+
+@pytest.fixture(scope="module")
+def pr1():
+    return gen_workload("pr1")
+
+
+@pytest.fixture(scope="module")
+def decode_small():
+    # decode's value distribution (outlier columns and channels) at a size
+    # the pure-numpy checks finish quickly
+    return gen_workload("decode", m=3, n=40, k=1280, seed=101)
+
+
+def test_transform_pins():
+    pins.check_transform(oracle.fwht128_f32, oracle.hadamard128)
+
+
+def test_transform_rounding_bound():
+    pins.check_transform_rounding(oracle.fwht128_f32)
+
+
+def test_transform_f64_matches_scipy():
+    x = np.random.default_rng(3).standard_normal((5, 256))
+    import scipy.linalg
+    H = scipy.linalg.hadamard(128).astype(np.float64)
+    ref = (x.reshape(5, 2, 128) @ H.T).reshape(5, 256)
+    assert np.allclose(oracle.fwht128_f64(x), ref, rtol=0, atol=1e-12)
+
+
+def test_transform_f32_exact_on_small_integers():
+    v = np.random.default_rng(5).integers(-1000, 1001, size=(8, 256)).astype(np.float32)
+    assert np.array_equal(oracle.fwht128_f32(v).astype(np.float64), oracle.fwht128_f64(v))
+
+
+def test_bf16_round_nearest_matches_torch():
+    rng = np.random.default_rng(9)
+    v = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * np.float32(37.0),
+        np.float32(2.0 ** -130) * rng.standard_normal(2000).astype(np.float32),  # bf16 subnormals
+        np.array([0.0, -0.0, 1.0, 1.00390625, 1.01171875, 3.3895e38, -3.3896e38], np.float32),
+    ])
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = oracle.bf16_round_nearest(v.astype(np.float64))
+    assert np.array_equal(got, ref)
+
+
+def test_bf16_round_up_is_smallest_upper_bound():
+    rng = np.random.default_rng(10)
+    v = np.abs(rng.standard_normal(20000).astype(np.float32)) * np.float32(1e-3)
+    v = np.concatenate([v, np.float32(2.0 ** -128) * np.abs(rng.standard_normal(500)).astype(np.float32),
+                        np.array([0.0, 1.0, 2.0 ** -126, 1.0078125], np.float32)])
+    r = oracle.bf16_round_up(v)
+    rb = r.view(np.uint32)
+    assert not np.any(rb & 0xFFFF)                      # on the bf16 grid
+    assert np.all(r >= v)                               # an upper bound
+    below = ((rb >> 16) - 1).astype(np.uint32) << 16    # next bf16 down
+    pos = r > 0
+    assert np.all(below[pos].view(np.float32) < v[pos])  # and the smallest one
+    assert np.all(r[v == 0] == 0)
+
+
+def test_act_golden():
+    pins.check_act_golden(oracle.act_quant)
+
+
+def test_act_properties(pr1, decode_small):
+    pins.check_act_properties(oracle.act_quant, oracle.fwht128_f64, pr1[0])
+    pins.check_act_properties(oracle.act_quant, oracle.fwht128_f64, decode_small[0])
+
+
+def test_act_spike_and_zero_rows():
+    pins.check_act_spike(oracle.act_quant)
+
+
+def test_act_unrotated_is_plain_absmax():
+    x = np.zeros((1, 128), np.float32)
+    x[0, :4] = [1.0, -0.5, 0.25, 2.0]
+    q, a = oracle.act_quant(pins.bf16(x).reshape(1, 128), rotate=False)
+    assert list(q[0, :4]) == [64, -32, 16, 127] and np.all(q[0, 4:] == 0)  # 127/2 * x, ties to even
+    assert a[0] == np.float32(2.0) / np.float32(127.0)
+
+
+def test_pack_golden():
+    pins.check_pack_golden(oracle.pack)
+
+
+def test_pack_g256_properties(pr1, decode_small):
+    pins.check_pack_g256_properties(oracle.pack, oracle.fwht128_f64, pr1[1])
+    pins.check_pack_g256_properties(oracle.pack, oracle.fwht128_f64, decode_small[1])
+
+
+def test_pack_g128_properties(decode_small):
+    pins.check_pack_g128_properties(oracle.pack, oracle.fwht128_f64, decode_small[1])
+
+
+def test_pack_zero_row_and_sizes():
+    w = np.zeros((2, 512), np.uint16)
+    w[1] = pins.bf16(np.full(512, 0.25, np.float32))
+    codes, s1, s2 = oracle.pack(w, "g256", True)
+    assert s2[0] == 0 and np.all(s1[0] == 0) and np.all(codes[0] == 0)
+    assert s2[1] != 0
+    assert oracle.packed_sizes("g256", 17408, 5120) == (89128960, 348160, 34816)
+    assert oracle.packed_sizes("g128", 151936, 5120) == (777912320, 0, 12154880)
+    g = pins.golden("format")
+    assert g["trunk"]["group"] == oracle.GROUP_TRUNK and g["lm_head"]["group"] == oracle.GROUP_HEAD
+    assert g["trunk"]["code_max"] == oracle.CODE_MAX == -g["trunk"]["code_min"]
+
+
+def test_partials_brute_force():
+    rng = np.random.default_rng(12)
+    xq = rng.integers(-127, 128, size=(2, 512)).astype(np.int8)
+    codes = rng.integers(-127, 128, size=(3, 512)).astype(np.int8)
+    pins.check_partials_brute(oracle.partials, xq, codes, 256)
+    pins.check_partials_brute(oracle.partials, xq, codes, 128)
+    # extreme values: |P| reaches 256 * 127^2 exactly
+    full = np.full((1, 256), 127, np.int8)
+    assert oracle.partials(full, -full, 256)[0, 0, 0] == -256 * 127 * 127
+
+
+def test_linear_golden():
+    pins.check_linear_golden(oracle.act_quant, oracle.pack, oracle.partials, oracle.linear, oracle.linear_bf16)
+
+
+def test_product_identity_trunk(pr1, decode_small):
+    pins.check_product_identity(oracle.act_quant, oracle.pack, oracle.linear, pr1[0], pr1[1], "g256")
+    pins.check_product_identity(oracle.act_quant, oracle.pack, oracle.linear, decode_small[0], decode_small[1], "g256")
+
+
+def test_product_identity_lm_head():
+    x, w = gen_workload("lm_head8", m=2, n=48, k=640, seed=104)
+    pins.check_product_identity(oracle.act_quant, oracle.pack, oracle.linear, x, w, "g128")
+
+
+def test_unrotated_linear_is_plain_int8_linear(pr1):
+    x, w = pr1
+    xq, a = oracle.act_quant(x, rotate=False)
+    codes, s1, s2 = oracle.pack(w, "g256", rotate=False)
+    y = oracle.linear(xq, a, "g256", codes, s1, s2, rotated=False)
+    ref = (a.astype(np.float64)[:, None] * xq.astype(np.float64)) @ (
+        np.repeat(pins.bf16_val(s2).astype(np.float64)[:, None] * s1, 256, axis=1) * codes).T
+    assert np.allclose(y, ref, rtol=1e-12, atol=0)
+
+
+def test_rotated_and_unrotated_agree(pr1):
+    x, w = pr1
+    ys = []
+    for rot in (True, False):
+        xq, a = oracle.act_quant(x, rotate=rot)
+        codes, s1, s2 = oracle.pack(w, "g256", rotate=rot)
+        ys.append(oracle.linear(xq, a, "g256", codes, s1, s2, rotated=rot))
+    assert np.sqrt(np.mean((ys[0] - ys[1]) ** 2)) < 0.05 * np.sqrt(np.mean(ys[1] ** 2))
+
+
+def test_workload_shapes_cover_the_pages_sizes():
+    assert (WORKLOADS["decode"].k, WORKLOADS["decode"].n) == (5120, 17408)
+    assert (WORKLOADS["verify128"].k, WORKLOADS["verify128"].n) == (17408, 5120)
+    assert WORKLOADS["prefill"].m == 8192 and WORKLOADS["lm_head1"].n == 151936

@@ -1,0 +1,134 @@
+"""Plant plausible mistakes in the oracle (CPU only) and check a pin fails.
+
+Each mutation is patched into the oracle module for the duration of one test,
+so the oracle's own functions run with the mistake inside them.
+"""
+
+import types
+
+import numpy as np
+import pytest
+
+import oracle
+import oracle.iq8r_oracle as om
+import pins
+from iq8r_inputs import gen_workload
+
+X, W = gen_workload("decode", m=3, n=40, k=1280, seed=101)
+
+
+def np_proxy(**overrides):
+    """A stand-in for the numpy module with some functions replaced."""
+    ns = types.SimpleNamespace(**{k: getattr(np, k) for k in dir(np) if not k.startswith("__")})
+    for k, v in overrides.items():
+        setattr(ns, k, v)
+    return ns
+
+
+def fwht_sign_flipped(v):
+    v = np.asarray(v, dtype=np.float32)
+    x = v.reshape(-1, 128).copy()
+    h = 1
+    while h < 128:
+        y = x.reshape(x.shape[0], 128 // (2 * h), 2, h)
+        lo, hi = y[:, :, 0, :].copy(), y[:, :, 1, :].copy()
+        y[:, :, 0, :] = lo - hi
+        y[:, :, 1, :] = lo + hi
+        h *= 2
+    return x.reshape(v.shape)
+
+
+def fwht_missing_stage(v):
+    v = np.asarray(v, dtype=np.float32)
+    x = v.reshape(-1, 128).copy()
+    h = 1
+    while h < 64:
+        y = x.reshape(x.shape[0], 128 // (2 * h), 2, h)
+        lo, hi = y[:, :, 0, :].copy(), y[:, :, 1, :].copy()
+        y[:, :, 0, :] = lo + hi
+        y[:, :, 1, :] = lo - hi
+        h *= 2
+    return x.reshape(v.shape)
+
+
+def nearest_bf16_not_up(v):
+    b = om.bf16_round_nearest(np.asarray(v, dtype=np.float64))
+    return (b.astype(np.uint32) << 16).view(np.float32)
+
+
+def fails(check):
+    with pytest.raises(AssertionError):
+        check()
+
+
+@pytest.mark.parametrize("bad", [fwht_sign_flipped, fwht_missing_stage])
+def test_broken_butterfly_is_caught(monkeypatch, bad):
+    monkeypatch.setattr(om, "fwht128_f32", bad)
+    fails(lambda: pins.check_transform(om.fwht128_f32, om.hadamard128))
+    fails(lambda: pins.check_act_spike(om.act_quant))
+
+
+def test_floor_instead_of_rint_is_caught(monkeypatch):
+    monkeypatch.setattr(om, "np", np_proxy(rint=np.floor))
+    fails(lambda: pins.check_act_properties(om.act_quant, om.fwht128_f64, X))
+    fails(lambda: pins.check_pack_g256_properties(om.pack, om.fwht128_f64, W))
+
+
+def test_floor_instead_of_ceil_for_sub_scale_is_caught(monkeypatch):
+    monkeypatch.setattr(om, "np", np_proxy(ceil=np.floor))
+    fails(lambda: pins.check_pack_g256_properties(om.pack, om.fwht128_f64, W))
+
+
+def test_nearest_instead_of_round_up_scale_is_caught(monkeypatch):
+    monkeypatch.setattr(om, "bf16_round_up", nearest_bf16_not_up)
+    fails(lambda: pins.check_pack_golden(om.pack))
+
+
+def test_wrong_activation_divisor_is_caught(monkeypatch):
+    real = om.act_quant
+
+    def act_128(x_bits, rotate=True):
+        # codes on a 128-level grid while a still says amax / 127
+        q, a = real(x_bits, rotate)
+        xr = om.fwht128_f32(om.bf16_to_f32(x_bits))
+        amax = np.abs(xr).max(axis=1)
+        q = np.clip(np.rint(xr * (np.float32(128) / amax)[:, None]), -127, 127).astype(np.int8)
+        return q, a
+
+    fails(lambda: pins.check_act_properties(act_128, om.fwht128_f64, X))
+
+
+def test_dropped_output_factor_is_caught():
+    def linear_no_128(*args, **kw):
+        kw["rotated"] = False
+        return oracle.linear(*args, **kw)
+
+    fails(lambda: pins.check_product_identity(oracle.act_quant, oracle.pack, linear_no_128, X, W, "g256"))
+
+
+def test_misindexed_sub_scale_is_caught():
+    def pack_reversed_s1(w_bits, fmt, rotate=True):
+        codes, s1, s2 = oracle.pack(w_bits, fmt, rotate)
+        return codes, s1[:, ::-1].copy(), s2
+
+    fails(lambda: pins.check_product_identity(oracle.act_quant, pack_reversed_s1, oracle.linear, X, W, "g256"))
+
+
+def test_shifted_block_boundary_is_caught():
+    def partials_shifted(xq, codes, group):
+        return oracle.partials(np.roll(xq, 1, axis=1), codes, group)
+
+    rng = np.random.default_rng(12)
+    xq = rng.integers(-127, 128, size=(2, 512)).astype(np.int8)
+    codes = rng.integers(-127, 128, size=(3, 512)).astype(np.int8)
+    fails(lambda: pins.check_partials_brute(partials_shifted, xq, codes, 256))
+
+
+def test_transposed_weight_blocks_are_caught():
+    def pack_swapped_halves(w_bits, fmt, rotate=True):
+        codes, s1, s2 = oracle.pack(w_bits, fmt, rotate)
+        n, k = codes.shape
+        c = codes.reshape(n, k // 256, 256)[:, ::-1].reshape(n, k).copy()
+        return c, s1, s2
+
+    fails(lambda: pins.check_product_identity(oracle.act_quant, pack_swapped_halves, oracle.linear, X, W, "g256"))
