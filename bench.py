@@ -1,0 +1,502 @@
+#!/usr/bin/env python
+"""Benchmark of the IQ8R rotated W8A8 linear (libiq8r) on B200.
+
+A step is one pass of the whole hot path over one batch: rotate + int8
+quantise the activations (iq8r_rotate_quant_act), then the int8 linear with
+its fused scale epilogue (iq8r_linear). The default workload is the decode
+GEMV (M=1, K=5120, N=17408, trunk format); --config picks another.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode]
+    python bench.py --impl reference ...   # the CPU oracle, same metric
+
+Timing: inputs resident in HBM; several weight copies are rotated so that
+the bytes touched between two uses of a copy exceed 3x L2 (or one copy when
+a step alone moves more than that); the K steps replay CUDA graphs on one
+stream, bracketed by a barrier and synchronize; per-kernel durations come
+from CUDA events recorded inside the same graphs. Multi-GPU runs are
+independent replicas (one process per GPU, no data-path collective): the
+whole-job value is the units all ranks processed over the slowest rank's
+time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "IQ8R W8A8 linear: decode HBM GB/s and prefill int8 TOPS vs B200 peak"
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+INT8_OVER_BF16 = 2.0  # nominal dense ratio (4.5 POPS int8 / 2.25 PFLOP/s bf16)
+
+CONFIGS = {
+    # name: (m, k, n, fmt, default steps)
+    "pr1": (4, 512, 256, "g256", 2000),
+    "decode": (1, 5120, 17408, "g256", 20000),
+    "verify8": (8, 17408, 5120, "g256", 5000),
+    "verify16": (16, 17408, 5120, "g256", 2000),
+    "verify128": (128, 17408, 5120, "g256", 500),
+    "prefill": (8192, 5120, 17408, "g256", 20),
+    "lm_head1": (1, 5120, 151936, "g128", 2000),
+    "lm_head8": (8, 5120, 151936, "g128", 1000),
+}
+
+
+# ------------------------------------------------------------------ bytes
+
+def act_bytes(m, k):
+    """Rotate-quantise: bf16 in, int8 codes and one fp32 scale per token out."""
+    return 2 * m * k + m * k + 4 * m
+
+
+def linear_bytes(m, k, n, fmt):
+    """Weights (codes + scales), int8 activations + scales in, bf16 out."""
+    if fmt == "g256":
+        w = n * k + n * (k // 256) + 2 * n
+    else:
+        w = n * k + 2 * n * (k // 128)
+    return w + m * k + 4 * m + 2 * m * n
+
+
+def step_bytes(m, k, n, fmt):
+    return act_bytes(m, k) + linear_bytes(m, k, n, fmt)
+
+
+# ------------------------------------------------------------------ peaks
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def kernel_source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, "quantised_fwht128_act_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel, workload, files):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel's
+    sources are unchanged since it was taken; else None."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        e = d[kernel][workload]
+        if e.get("source_hash") != kernel_source_hash(files):
+            return None
+        return int(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples (every 100 ms) while the benchmark runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.idx = device_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.idx)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+
+    def summary(self, t0, t1):
+        def num(s):
+            try:
+                return float(s)
+            except ValueError:
+                return None
+
+        inside = [p for t, p in self.samples if t0 <= t <= t1]
+        window = "timed region"
+        if not inside:
+            inside = [p for _, p in self.samples]
+            window = "whole run (the timed region was shorter than one sample)"
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "window": "no nvidia-smi"}
+        sm = [num(p[1]) for p in inside if num(p[1]) is not None]
+        smax = [num(p[2]) for p in inside if num(p[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for p in inside for i in range(4) if p[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(inside), "window": window}
+
+
+# ------------------------------------------------------------- workload
+
+def make_inputs(cfg_name, copies_hint=None):
+    """Host inputs: x copies (bf16 bits) and the packed weight (host packer)."""
+    import quantised_fwht128_act_b200 as iq8r
+    from iq8r_inputs import WORKLOADS, f32_to_bf16_bits, gen_act, gen_workload
+    m, k, n, fmt, _ = CONFIGS[cfg_name]
+    wl = WORKLOADS.get(cfg_name, WORKLOADS["decode"])
+    x0, w = gen_workload(wl, m=m, n=n, k=k)
+    packed = iq8r.iq8r_pack(w, fmt, True)
+    del w
+    return x0, packed, wl
+
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import quantised_fwht128_act_b200 as iq8r
+    from iq8r_inputs import f32_to_bf16_bits, gen_act
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    m, k, n, fmt, _ = CONFIGS[args.config]
+    K, W = args.steps, args.warmup
+    x0, (codes, sub, scale), wl = make_inputs(args.config)
+
+    # rotating copies so that consecutive uses of one copy are > 3x L2 apart
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    footprint = step_bytes(m, k, n, fmt)
+    R = 1 if footprint > 3 * l2 else int(math.ceil(3 * l2 / footprint)) + 1
+    weights = []
+    base = iq8r.IQ8RWeight.from_packed(codes, sub, scale, fmt, True, device=dev)
+    weights.append(base)
+    for _ in range(R - 1):
+        weights.append(iq8r.IQ8RWeight(base.fmt, base.rotated, base.n, base.k, base.codes.clone(),
+                                       None if base.sub_scale is None else base.sub_scale.clone(),
+                                       base.scale.clone()))
+    rng = np.random.default_rng(1000 + rank)
+    xs_host = [x0] + [f32_to_bf16_bits(gen_act(rng, m, k, wl.x_outliers, wl.x_outlier_mult)) for _ in range(R - 1)]
+    x_dev = [torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16) for x in xs_host]
+    xq = [torch.empty((m, k), dtype=torch.int8, device=dev) for _ in range(R)]
+    xsc = [torch.empty((m,), dtype=torch.float32, device=dev) for _ in range(R)]
+    y = [torch.empty((m, n), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    launches_per_step = 2 + (0 if m <= 8 else (m + 7) // 8 - 1)  # act + GEMV groups of 8 tokens
+
+    def step(j):
+        r = j % R
+        iq8r.iq8r_rotate_quant_act(x_dev[r], True, xq[r], xsc[r])
+        iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for j in range(max(W, 1)):
+            step(j)
+    stream.synchronize()
+    iq8r.iq8r_get_device_error(stream)
+
+    # graphs: a main chunk of C steps (a multiple of R) and a tail, each step
+    # bracketed by external events so the graph records kernel timestamps
+    C = min(K, max(R, (512 // R) * R))
+    n_main, tail = divmod(K, C)
+
+    def capture(nsteps, offset):
+        g = torch.cuda.CUDAGraph()
+        evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)] for _ in range(nsteps)]
+        with torch.cuda.graph(g, stream=stream):
+            for j in range(nsteps):
+                r = (offset + j) % R
+                evs[j][0].record()
+                iq8r.iq8r_rotate_quant_act(x_dev[r], True, xq[r], xsc[r])
+                evs[j][1].record()
+                iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
+                evs[j][2].record()
+        return g, evs
+
+    g_main, ev_main = capture(C, 0) if n_main else (None, None)
+    g_tail, ev_tail = capture(tail, 0) if tail else (None, None)
+    # one untimed replay of each graph (upload, first-touch)
+    for g in (g_main, g_tail):
+        if g is not None:
+            with torch.cuda.stream(stream):
+                g.replay()
+    stream.synchronize()
+
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start_wall = time.time()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record()
+        for _ in range(n_main):
+            g_main.replay()
+        if g_tail is not None:
+            g_tail.replay()
+        end.record()
+    stream.synchronize()
+    torch.cuda.synchronize()
+    t_end_wall = time.time()
+    if world > 1:
+        torch.distributed.barrier()
+    time.sleep(0.25)
+    sampler.stop()
+    iq8r.iq8r_get_device_error(stream)
+
+    elapsed_ms = start.elapsed_time(end)
+    evs = ev_main if ev_main is not None else ev_tail
+    act_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    lin_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    del g_main, g_tail
+
+    # end to end through the public API: pinned H2D of x, the two calls,
+    # D2H of y, every step, eager launches
+    e2e = None
+    if not args.no_e2e:
+        xh = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in xs_host]
+        yh = [torch.empty((m, n), dtype=torch.bfloat16).pin_memory() for _ in range(R)]
+        xin = [torch.empty((m, k), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+        Ke = K
+        with torch.cuda.stream(stream):
+            for j in range(min(W, 50)):
+                r = j % R
+                xin[r].copy_(xh[r], non_blocking=True)
+                iq8r.iq8r_rotate_quant_act(xin[r], True, xq[r], xsc[r])
+                iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
+                yh[r].copy_(y[r], non_blocking=True)
+        stream.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        s0 = torch.cuda.Event(enable_timing=True)
+        s1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            s0.record()
+            for j in range(Ke):
+                r = j % R
+                xin[r].copy_(xh[r], non_blocking=True)
+                iq8r.iq8r_rotate_quant_act(xin[r], True, xq[r], xsc[r])
+                iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
+                yh[r].copy_(y[r], non_blocking=True)
+            s1.record()
+        stream.synchronize()
+        e_ms = s0.elapsed_time(s1)
+        if world > 1:
+            t = torch.tensor([e_ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": world * step_bytes(m, k, n, fmt) * Ke / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+               "h2d_bytes_per_step": 2 * m * k, "d2h_bytes_per_step": 2 * m * n, "steps": Ke,
+               "ms_per_step": e_ms / Ke, "how": "eager public-API calls on one stream, pinned host buffers"}
+
+    hbm, bf16_tf, peak_src = peaks()
+    lin_avg_ms = float(np.mean(lin_ms))
+    act_avg_ms = float(np.mean(act_ms))
+    lin_b = linear_bytes(m, k, n, fmt)
+    kern_files = ["gemv.cuh", "iq8r_device.cuh"]
+    if m <= 8:
+        achieved = lin_b / (lin_avg_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": "gemv_kernel", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "peak_source": f"{peak_src} HBM copy (MEASURED_PEAKS.json hbm_gbs)"
+                if peak_src == "measured" else "fallback 6.65 TB/s",
+                "traffic": recorded_traffic("gemv_kernel", args.config, kern_files),
+                "algorithmic_bytes_per_launch": lin_b, "avg_launch_ms": lin_avg_ms}
+    else:
+        ops = 2.0 * m * n * k
+        achieved_b = lin_b / (lin_avg_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "kernel": "gemv_kernel (token groups of 8)", "achieved": achieved_b, "peak": hbm,
+                "unit": "GB/s", "frac": achieved_b / hbm,
+                "int8_tops": ops / (lin_avg_ms * 1e-3) / 1e12,
+                "traffic": recorded_traffic("gemv_kernel", args.config, kern_files),
+                "algorithmic_bytes_per_launch": lin_b, "avg_launch_ms": lin_avg_ms}
+    roof["act_kernel"] = {"avg_launch_ms": act_avg_ms, "bytes": act_bytes(m, k),
+                          "achieved_gbs": act_bytes(m, k) / (act_avg_ms * 1e-3) / 1e9}
+
+    value = world * step_bytes(m, k, n, fmt) * K / (elapsed_ms * 1e-3) / 1e9
+    clocks = sampler.summary(t_start_wall, t_end_wall)
+    out = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8", "data": "synthetic",
+        "config": {"workload": args.config, "m": m, "k": k, "n": n, "format": fmt, "rotated": True,
+                   "step": "iq8r_rotate_quant_act + iq8r_linear",
+                   "bytes_per_step": step_bytes(m, k, n, fmt),
+                   "l2": f"{R} rotating weight/input copies ({R * footprint / 1e6:.0f} MB > 3x L2)" if R > 1
+                   else "a step moves more than 3x L2",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "timing": "CUDA graphs of the K steps; events inside the graphs time each kernel"},
+        "roofline": roof,
+        "clocks": clocks,
+        "gpu_launches": launches_per_step * K,
+        "e2e": e2e,
+        "cpu_baseline": None,
+    }
+    return out
+
+
+# ------------------------------------------------------------ CPU oracle
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def run_oracle(cfg_name, budget_s, steps=None):
+    """Time the oracle (as it stands) on a bounded sample of the workload.
+
+    A sample step is the oracle's act_quant over all M tokens plus its
+    linear over a slice of the N weight rows, sized to the budget. Returns
+    (value in GB/s of algorithmic bytes, sample description, steps, s/step).
+    """
+    import oracle
+    from iq8r_inputs import WORKLOADS, gen_workload
+    m, k, n, fmt, _ = CONFIGS[cfg_name]
+    wl = WORKLOADS.get(cfg_name, WORKLOADS["decode"])
+    m_s = min(m, 64)
+    n_probe = min(n, 256)
+    x, w = gen_workload(wl, m=m_s, n=n_probe, k=k)
+    packed = oracle.pack(w, fmt, True)
+    t = time.perf_counter()
+    q, a = oracle.act_quant(x)
+    oracle.linear(q, a, fmt, *packed, rotated=True)
+    probe = time.perf_counter() - t
+    per_row = probe / n_probe
+    if steps is None:
+        n_s = int(min(n, max(8, budget_s / 5 / max(per_row, 1e-9))))
+        reps = max(1, int(budget_s / max(per_row * n_s, 1e-9)))
+    else:
+        n_s = int(min(n, max(8, budget_s / steps / max(per_row, 1e-9))))
+        reps = steps
+    x, w = gen_workload(wl, m=m_s, n=n_s, k=k)
+    packed = oracle.pack(w, fmt, True)
+    del w
+    t = time.perf_counter()
+    for _ in range(reps):
+        q, a = oracle.act_quant(x)
+        oracle.linear(q, a, fmt, *packed, rotated=True)
+    dt = time.perf_counter() - t
+    b = step_bytes(m_s, k, n_s, fmt)
+    sample = (f"{reps} oracle steps of act_quant over {m_s} tokens + linear over {n_s} of {n} weight rows "
+              f"(K={k}, {fmt}); value = algorithmic bytes of that slice per second")
+    return b * reps / dt / 1e9, sample, reps, dt / reps
+
+
+def run_reference(args, rank, world):
+    m, k, n, fmt, _ = CONFIGS[args.config]
+    K, W = args.steps, args.warmup
+    budget = float(os.environ.get("IQ8R_REF_BUDGET_S", "60"))
+    # warm-up: W oracle steps of the same slice, untimed, within the budget
+    run_oracle(args.config, min(budget / 10, 5.0), steps=max(1, min(W, 3)))
+    value, sample, reps, s_per = run_oracle(args.config, budget, steps=K)
+    cores = blas_threads()
+    return {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": s_per * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8", "data": "synthetic", "impl": "reference",
+        "config": {"workload": args.config, "m": m, "k": k, "n": n, "format": fmt, "rotated": True},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------------ main
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", choices=sorted(CONFIGS), default="decode")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.steps is None:
+        args.steps = CONFIGS[args.config][4]
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        out = run_reference(args, rank, world)
+        print(json.dumps(out), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
+            value, sample, reps, _ = run_oracle(args.config, args.cpu_budget_s)
+            out["cpu_baseline"] = {"value": value, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+                                   "sample": sample}
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,179 @@
+/*
+ * libiq8r -- the IQ8R rotated W8A8 linear layer on NVIDIA B200 (sm_100a).
+ *
+ * The layer, as the "radiance" model cards describe it:
+ *
+ *  - "Qwen3.8-27B IQ8R + DFlash2 -- radiance container", table row "Weights":
+ *    every trunk linear is int8 with codes -127..127, a u8 scale per row and
+ *    256 of K under a bf16 scale per row, each 128 of K rotated by the
+ *    unnormalised Hadamard; the lm_head is int8 with a bf16 scale per row and
+ *    128 of K.
+ *  - same page, table row "Activations": int8 under the same rotation (W8A8).
+ *  - same page, "How this file was made": the recipe rules
+ *    "codes=i8 group=256 scale=u8 scale2=bf16 block2=1x* transform=fwht128
+ *    clamp=sym" (trunk) and "codes=i8 group=128 scale=bf16 clamp=sym"
+ *    (lm_head).
+ *
+ * Notation. W is a bf16 weight [N][K] (out x in), x a bf16 activation [M][K],
+ * H the 128x128 Sylvester Hadamard matrix (H[i][j] = (-1)^popcount(i&j),
+ * unnormalised, H H = 128 I), T(.) applies H to every consecutive 128 of K.
+ * y = x W^T is computed as (1/128) T(x) T(W)^T on int8 codes.
+ *
+ * Where the pages are silent the library follows stated definitions:
+ *  - the fp32 transform runs radix-2 butterflies h = 1, 2, ..., 64 in that
+ *    order, (a, b) -> (a + b, a - b), round-to-nearest-even, no fused ops;
+ *  - activations carry one fp32 scale per token: a = amax / 127,
+ *    codes = clamp(rint(x' * (127 / amax)), -127, 127);
+ *  - trunk weights: step d[n][g] = s2[n] * s1[n][g], s2 = bf16 of
+ *    R[n] / 32385 rounded up (R = row absmax of T(W)), s1 = min(255,
+ *    ceil(A[n][g] / (127 * s2))) (A = absmax of the 256-block);
+ *  - lm_head weights: s[n][g] = bf16 of A[n][g] / 127 rounded up;
+ *  - round-half-to-even wherever a value is rounded to nearest.
+ *
+ * Conventions for every call:
+ *  - The caller owns every buffer. Hot calls allocate nothing.
+ *  - Device pointers must be device memory of the current CUDA device and
+ *    16-byte aligned; tensors are dense and row-major as stated.
+ *  - A bad argument returns IQ8R_ERR_INVALID_ARG, launches nothing and sets
+ *    the thread's message (iq8r_last_error). A failed launch returns
+ *    IQ8R_ERR_CUDA.
+ *  - GPU calls are asynchronous and ordered on `stream` (0 = the legacy
+ *    default stream). Kernels never trap: a bounded wait that runs out sets
+ *    a device error word that iq8r_get_device_error reports.
+ */
+#ifndef IQ8R_H_
+#define IQ8R_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  IQ8R_OK = 0,
+  IQ8R_ERR_INVALID_ARG = 1,    /* bad shape, pointer, alignment or format */
+  IQ8R_ERR_UNSUPPORTED = 2,    /* valid request this build cannot serve */
+  IQ8R_ERR_CUDA = 3,           /* a CUDA runtime call or launch failed */
+  IQ8R_ERR_DEVICE_TIMEOUT = 4  /* a kernel's bounded wait ran out */
+} iq8r_status;
+
+typedef enum {
+  /* trunk: int8 codes, u8 sub-scale per (row, 256 of K), bf16 scale per row */
+  IQ8R_FMT_G256_U8_BF16 = 0,
+  /* lm_head: int8 codes, bf16 scale per (row, 128 of K) */
+  IQ8R_FMT_G128_BF16 = 1
+} iq8r_format;
+
+/* Kernel choice for iq8r_linear_ex. AUTO picks by M. */
+typedef enum {
+  IQ8R_PATH_AUTO = 0,
+  IQ8R_PATH_GEMV = 1,   /* weight-streaming dp4a GEMV, M handled 8 rows at a time */
+  IQ8R_PATH_TC = 2      /* tcgen05 kind::i8 tensor-core GEMM */
+} iq8r_path;
+
+/* A packed weight on the device. Not owned by the library.
+ *   codes     int8 [n][k], K contiguous (row-major), values -127..127
+ *   sub_scale u8   [n][k/256] for IQ8R_FMT_G256_U8_BF16; NULL for G128
+ *   scale     bf16 [n] (G256) or [n][k/128] (G128), as raw 16-bit patterns
+ *   rotated   1 if the codes live in the fwht128 domain (the output is then
+ *             multiplied by 1/128); 0 for a plain int8 weight.
+ * k must be a multiple of 256 (G256) or 128 (G128); codes and scale must be
+ * 16-byte aligned; sub_scale needs no alignment. */
+typedef struct {
+  int32_t fmt;
+  int32_t rotated;
+  int64_t n;
+  int64_t k;
+  const int8_t* codes;
+  const uint8_t* sub_scale;
+  const uint16_t* scale;
+} iq8r_weight;
+
+/* Byte sizes of the three packed arrays for an [n][k] weight of `fmt`
+ * (sub_bytes is 0 for G128). Host only; any pointer may be NULL. */
+iq8r_status iq8r_packed_sizes(int32_t fmt, int64_t n, int64_t k, size_t* codes_bytes,
+                              size_t* sub_bytes, size_t* scale_bytes);
+
+/* Round-to-nearest packing of a bf16 weight (the recipes' "rtn"; the pages'
+ * own GPTQ fit needs calibration Hessians and is not part of this library).
+ * Host memory in and out, synchronous.
+ *   w_bf16    bf16 [n][k] host, raw 16-bit patterns
+ *   rotate    1: apply fwht128 to each 128 of K first (k % 128 == 0)
+ *   codes     int8 [n][k] host (out)
+ *   sub_scale u8 [n][k/256] host (out; G256 only, NULL for G128)
+ *   scale     bf16 [n] (G256) or [n][k/128] (G128) host (out)
+ *   n_threads host threads to use; <= 0 picks the hardware concurrency.
+ * Trunk: "a u8 scale per row and 256 of K under a bf16 scale a row" (IQ8R
+ * page, "Weights"); lm_head: "a bf16 scale per row and 128" (same row).
+ * Output is byte-identical to the stated definition in the file comment. */
+iq8r_status iq8r_pack(int32_t fmt, int32_t rotate, const uint16_t* w_bf16, int64_t n, int64_t k,
+                      int8_t* codes, uint8_t* sub_scale, uint16_t* scale, int32_t n_threads);
+
+/* Rotate and quantise activations: "int8 under the same rotation (W8A8)"
+ * (IQ8R page, "Activations"), one fp32 scale per token.
+ *   x_bf16  device bf16 [m][k], raw 16-bit patterns, 16-byte aligned
+ *   m >= 0 (0 launches nothing), k % 128 == 0, 0 < k <= 2^30
+ *   rotate  1: x' = T(x) in fp32; 0: x' = x
+ *   xq      device int8 [m][k] (out), 16-byte aligned
+ *   x_scale device fp32 [m] (out): a = amax(|x'|) / 127 (0 for a zero row)
+ * Codes and scales are bit-identical to the stated definition. */
+iq8r_status iq8r_rotate_quant_act(const uint16_t* x_bf16, int64_t m, int64_t k, int32_t rotate,
+                                  int8_t* xq, float* x_scale, cudaStream_t stream);
+
+/* y = x W^T on int8 codes, the scale epilogue fused, bf16 out.
+ *   xq      device int8 [m][w->k] from iq8r_rotate_quant_act (same rotate
+ *           setting as the weight), 16-byte aligned
+ *   x_scale device fp32 [m]
+ *   m >= 0 (0 launches nothing)
+ *   y_bf16  device bf16 [m][w->n] (out), 16-byte aligned
+ * Trunk:   y[m][n] = bf16_rn(a[m] * s2[n] * sum_g s1[n][g] * P[m][n][g] / 128)
+ * lm_head: y[m][n] = bf16_rn(a[m] / 128 * sum_g s[n][g] * P[m][n][g])
+ * with P the exact int32 dot product of the codes over block g (256 or 128
+ * of K); /128 only when w->rotated. The sum over g is carried in fp32 or
+ * exact integers, so y matches the float64 value to within its bf16
+ * rounding plus ~1e-6 of the output's scale. */
+iq8r_status iq8r_linear(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,
+                        uint16_t* y_bf16, cudaStream_t stream);
+
+/* iq8r_linear with an explicit kernel choice (tests and measurement). */
+iq8r_status iq8r_linear_ex(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,
+                           uint16_t* y_bf16, int32_t path, cudaStream_t stream);
+
+/* Debug twin of iq8r_linear: writes the exact per-block int32 partial sums
+ * P[i][j][g] = sum_{k in block g} xq[i][k] * codes[n0 + j][k] for rows
+ * n0 <= n < n1 instead of y, computed by the same kernel code as the
+ * chosen path (0 <= n0 < n1 <= w->n; block = 256 for G256, 128 for G128).
+ *   p  device int32 [m][n1 - n0][k / block] (out), 16-byte aligned */
+iq8r_status iq8r_linear_partials(const int8_t* xq, int64_t m, const iq8r_weight* w, int64_t n0,
+                                 int64_t n1, int32_t* p, int32_t path, cudaStream_t stream);
+
+/* Synchronises `stream`, then reads and clears the current device's error
+ * word. IQ8R_OK if no kernel reported a problem since the last call;
+ * IQ8R_ERR_DEVICE_TIMEOUT if a bounded wait ran out (the message names the
+ * kernel and the wait); IQ8R_ERR_CUDA if the stream itself failed. */
+iq8r_status iq8r_get_device_error(cudaStream_t stream);
+
+/* Failure-path self-test (no counterpart on the pages). Launches one
+ * kernel whose bounded wait waits on a barrier that nothing arrives on, so
+ * it gives up after limit_ns (1e3..1e8 ns) and records a self-test code; the
+ * next iq8r_get_device_error then returns IQ8R_ERR_DEVICE_TIMEOUT and the
+ * context stays usable. It exercises the same wait that every pipelined
+ * kernel uses, without faulting or hanging the GPU. */
+iq8r_status iq8r_selftest_wait_timeout(int64_t limit_ns, cudaStream_t stream);
+
+/* The calling thread's message for its last failed call ("" if none).
+ * Valid until the thread's next libiq8r call. */
+const char* iq8r_last_error(void);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int32_t iq8r_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* IQ8R_H_ */

@@ -1,0 +1,170 @@
+// Activation rotate + int8 quantise: "int8 under the same rotation (W8A8)"
+// ("Qwen3.8-27B IQ8R + DFlash2 -- radiance container", table row
+// "Activations"), one fp32 scale per token.
+//
+// One CTA per token row. A thread owns "slots" of 16 consecutive elements
+// (two 16-byte bf16 loads, one 16-byte int8 store). A 128-chunk is 8 slots
+// held by 8 consecutive lanes, so fwht128's seven butterfly stages run as
+// h = 1, 2, 4, 8 inside the thread and h = 16, 32, 64 across lanes (xor 1,
+// 2, 4), in that order, each an IEEE add or subtract: the result is
+// bit-identical to the sequential radix-2 transform.
+#pragma once
+
+#include "iq8r_device.cuh"
+
+namespace iq8r {
+
+constexpr int kActSlot = 16;           // elements per slot
+constexpr int kActRegMaxK = 16384;     // register path up to this K
+constexpr int kActTwoPassThreads = 256;
+
+__device__ __forceinline__ void act_load_slot(const uint16_t* p, float (&v)[kActSlot], bool streaming) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+  uint4 lo, hi;
+  if (streaming) {
+    lo = __ldcs(q);
+    hi = __ldcs(q + 1);
+  } else {
+    lo = __ldg(q);
+    hi = __ldg(q + 1);
+  }
+  const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    v[2 * i] = __uint_as_float(w[i] << 16);
+    v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+  }
+}
+
+// fwht128 of the chunk this lane's slot belongs to (8 lanes per chunk).
+__device__ __forceinline__ void act_fwht_slot(float (&v)[kActSlot], int lane) {
+#pragma unroll
+  for (int h = 1; h < kActSlot; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < kActSlot; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i];
+        const float b = v[i + h];
+        v[i] = __fadd_rn(a, b);
+        v[i + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int b = 1; b < 8; b <<= 1) {
+    const bool upper = (lane & b) != 0;
+#pragma unroll
+    for (int i = 0; i < kActSlot; ++i) {
+      const float o = __shfl_xor_sync(0xffffffffu, v[i], b);
+      v[i] = upper ? __fsub_rn(o, v[i]) : __fadd_rn(v[i], o);
+    }
+  }
+}
+
+__device__ __forceinline__ float act_slot_absmax(const float (&v)[kActSlot]) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < kActSlot; ++i) m = fmaxf(m, fabsf(v[i]));
+  return m;
+}
+
+__device__ __forceinline__ void act_store_slot(int8_t* p, const float (&v)[kActSlot], float inv) {
+  uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int i = 0; i < kActSlot; ++i) {
+    int q = __float2int_rn(__fmul_rn(v[i], inv));
+    q = max(-127, min(127, q));
+    w[i >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (i & 3));
+  }
+  *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// CTA-wide max of non-negative floats; every thread gets the result.
+__device__ __forceinline__ float act_block_max(float v, float* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[warp] = v;
+  __syncthreads();
+  float m = 0.0f;
+  for (int w = 0; w < nwarps; ++w) m = fmaxf(m, red[w]);
+  return m;
+}
+
+// K <= kActRegMaxK: the row stays in registers (J slots per thread).
+template <int J>
+__global__ void __launch_bounds__(128) act_quant_reg_kernel(const uint16_t* __restrict__ x, int k, int rotate,
+                                                            int8_t* __restrict__ xq, float* __restrict__ xs) {
+  __shared__ float red[32];
+  const int64_t row = blockIdx.x;
+  const int slots = k / kActSlot;
+  const int lane = threadIdx.x & 31;
+  const uint16_t* xr = x + row * k;
+  float v[J][kActSlot];
+  float amax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int s = threadIdx.x + j * blockDim.x;
+    if (s < slots) {
+      act_load_slot(xr + s * kActSlot, v[j], true);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kActSlot; ++i) v[j][i] = 0.0f;
+    }
+    if (rotate) act_fwht_slot(v[j], lane);  // whole 8-lane groups are in or out
+    amax = fmaxf(amax, act_slot_absmax(v[j]));
+  }
+  amax = act_block_max(amax, red);
+  const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+  int8_t* qr = xq + row * k;
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int s = threadIdx.x + j * blockDim.x;
+    if (s < slots) act_store_slot(qr + s * kActSlot, v[j], inv);
+  }
+  if (threadIdx.x == 0) xs[row] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+}
+
+// Any K: pass 1 finds amax, pass 2 reloads the row (now in L2), repeats the
+// identical transform and quantises.
+__global__ void __launch_bounds__(kActTwoPassThreads) act_quant_2pass_kernel(const uint16_t* __restrict__ x, int k,
+                                                                             int rotate, int8_t* __restrict__ xq,
+                                                                             float* __restrict__ xs) {
+  __shared__ float red[32];
+  const int64_t row = blockIdx.x;
+  const int slots = k / kActSlot;
+  const int lane = threadIdx.x & 31;
+  const uint16_t* xr = x + row * static_cast<int64_t>(k);
+  const int iters = (slots + blockDim.x - 1) / blockDim.x;
+  float v[kActSlot];
+  float amax = 0.0f;
+  for (int j = 0; j < iters; ++j) {
+    const int s = threadIdx.x + j * blockDim.x;
+    if (s < slots) {
+      act_load_slot(xr + static_cast<int64_t>(s) * kActSlot, v, false);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kActSlot; ++i) v[i] = 0.0f;
+    }
+    if (rotate) act_fwht_slot(v, lane);
+    amax = fmaxf(amax, act_slot_absmax(v));
+  }
+  amax = act_block_max(amax, red);
+  const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+  int8_t* qr = xq + row * static_cast<int64_t>(k);
+  for (int j = 0; j < iters; ++j) {
+    const int s = threadIdx.x + j * blockDim.x;
+    if (s < slots) {
+      act_load_slot(xr + static_cast<int64_t>(s) * kActSlot, v, false);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kActSlot; ++i) v[i] = 0.0f;
+    }
+    if (rotate) act_fwht_slot(v, lane);
+    if (s < slots) act_store_slot(qr + static_cast<int64_t>(s) * kActSlot, v, inv);
+  }
+  if (threadIdx.x == 0) xs[row] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+}
+
+}  // namespace iq8r

@@ -1,0 +1,60 @@
+// Internal interface between the C ABI (iq8r_api.cpp, host C++) and the
+// CUDA launchers (iq8r_kernels.cu). Not installed; not part of the ABI.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <string>
+
+#include <cuda_runtime_api.h>
+
+namespace iq8r {
+
+constexpr int kGroupTrunk = 256;  // u8 sub-scale block of the trunk format
+constexpr int kGroupHead = 128;   // bf16 scale block of the lm_head format
+constexpr int kRot = 128;         // fwht128 acts on each 128 of K
+
+// Device error word values (0 = no error). The low byte names the wait.
+enum DeviceError : uint32_t {
+  kDevErrNone = 0,
+  kDevErrGemvFull = 0x101,    // GEMV consumer: weight stage never arrived
+  kDevErrGemvEmpty = 0x102,   // GEMV producer: ring slot never released
+  kDevErrGemvDrain = 0x103,   // GEMV producer: copy in flight at exit
+  kDevErrTcFull = 0x201,      // TC GEMM: operand stage never arrived
+  kDevErrTcEmpty = 0x202,     // TC GEMM: operand slot never released
+  kDevErrTcAccFull = 0x203,   // TC GEMM: accumulator never committed
+  kDevErrTcAccEmpty = 0x204,  // TC GEMM: accumulator never drained
+  kDevErrTcDrain = 0x205,     // TC GEMM: copy in flight at exit
+  kDevErrSelftest = 0x301,    // self-test wait that nothing satisfies
+};
+
+struct LinearArgs {
+  const int8_t* xq;      // [m][k]
+  const float* xs;       // [m]
+  int64_t m;
+  int fmt;               // 0 = G256 trunk, 1 = G128 lm_head
+  int rotated;
+  int64_t n;
+  int64_t k;
+  const int8_t* codes;   // [n][k]
+  const uint8_t* sub;    // [n][k/256] (G256)
+  const uint16_t* scale; // [n] (G256) or [n][k/128] (G128)
+  uint16_t* y;           // [m][n] bf16, or nullptr in partials mode
+  int32_t* partials;     // [m][n][k/G] in partials mode, else nullptr
+};
+
+// Launchers (iq8r_kernels.cu). They validate nothing: the ABI layer has.
+cudaError_t launch_act_quant(const uint16_t* x, int64_t m, int64_t k, int rotate, int8_t* xq,
+                             float* xs, cudaStream_t stream);
+cudaError_t launch_gemv(const LinearArgs& a, cudaStream_t stream);
+bool gemv_supported(int64_t k, std::string* why);
+cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream);
+bool gemm_tc_supported(const LinearArgs& a, std::string* why);
+cudaError_t read_and_clear_device_error(uint32_t* err);
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
+
+// Host packer (iq8r_pack.cpp).
+void pack_rows(int fmt, bool rotate, const uint16_t* w, int64_t n, int64_t k, int8_t* codes,
+               uint8_t* sub, uint16_t* scale, int n_threads);
+
+}  // namespace iq8r

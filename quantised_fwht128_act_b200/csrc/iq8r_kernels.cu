@@ -1,0 +1,213 @@
+// Launchers for the IQ8R kernels. All device code lives in this one
+// translation unit so the per-device error word is a single symbol.
+
+#include <algorithm>
+#include <atomic>
+#include <string>
+
+#include "act_quant.cuh"
+#include "gemv.cuh"
+#include "iq8r_device.cuh"
+#include "iq8r_internal.h"
+
+namespace iq8r {
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceInfo {
+  int num_sms = 0;
+  int smem_optin = 0;
+};
+
+DeviceInfo g_dev[kMaxDevices];
+std::atomic<int> g_dev_ready[kMaxDevices];
+
+cudaError_t device_info(DeviceInfo* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (g_dev_ready[dev].load(std::memory_order_acquire) == 0) {
+    DeviceInfo d;
+    e = cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&d.smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+    if (e != cudaSuccess) return e;
+    g_dev[dev] = d;
+    g_dev_ready[dev].store(1, std::memory_order_release);
+  }
+  *out = g_dev[dev];
+  return cudaSuccess;
+}
+
+// Raise a kernel's dynamic shared memory limit once per device (and again
+// only if a larger size is asked for).
+template <typename Kernel>
+cudaError_t ensure_smem(Kernel kernel, int bytes) {
+  static std::atomic<int> configured[kMaxDevices];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (configured[dev].load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) configured[dev].store(bytes, std::memory_order_release);
+  return e;
+}
+
+// Static shared memory and alignment slack kept out of the dynamic budget.
+constexpr int kSmemReserve = 1024;
+
+template <int MT, int FMT, bool PARTIALS>
+cudaError_t launch_gemv_t(const LinearArgs& a, const DeviceInfo& d, cudaStream_t stream) {
+  const int k = static_cast<int>(a.k);
+  const int red = gemv_red_bytes<MT, FMT>();
+  const int base = gemv_smem_bytes(MT, k, 0, red);
+  const int budget = d.smem_optin - kSmemReserve;
+  const int stages = std::min(kGemvMaxStages, (budget - base) / (kGemvStageBytes + 16));
+  if (stages < 2) return cudaErrorInvalidConfiguration;
+  const int smem = gemv_smem_bytes(MT, k, stages, red);
+  auto kernel = gemv_kernel<MT, FMT, PARTIALS>;
+  cudaError_t e = ensure_smem(kernel, smem);
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = (a.n + kGemvRows - 1) / kGemvRows;
+  const int64_t grid = std::min<int64_t>(d.num_sms, tiles);
+  kernel<<<static_cast<unsigned>(grid), kGemvThreads, smem, stream>>>(a, stages, tiles / grid, tiles % grid);
+  return cudaGetLastError();
+}
+
+template <int FMT, bool PARTIALS>
+cudaError_t launch_gemv_mt(const LinearArgs& a, int mt, const DeviceInfo& d, cudaStream_t stream) {
+  switch (mt) {
+    case 1: return launch_gemv_t<1, FMT, PARTIALS>(a, d, stream);
+    case 2: return launch_gemv_t<2, FMT, PARTIALS>(a, d, stream);
+    case 4: return launch_gemv_t<4, FMT, PARTIALS>(a, d, stream);
+    default: return launch_gemv_t<8, FMT, PARTIALS>(a, d, stream);
+  }
+}
+
+int next_pow2(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+// Largest token tile (1, 2, 4 or 8) whose activation codes leave room for a
+// two-stage ring.
+int gemv_max_mt(int64_t k, const DeviceInfo& d) {
+  for (int mt = 8; mt >= 1; mt >>= 1) {
+    const int need = gemv_smem_bytes(mt, static_cast<int>(k), 2, 2 * 8 * 8 * 8);
+    if (need <= d.smem_optin - kSmemReserve) return mt;
+  }
+  return 0;
+}
+
+}  // namespace
+
+cudaError_t launch_act_quant(const uint16_t* x, int64_t m, int64_t k, int rotate, int8_t* xq, float* xs,
+                             cudaStream_t stream) {
+  if (m == 0) return cudaSuccess;
+  const int slots = static_cast<int>(k / kActSlot);
+  const unsigned grid = static_cast<unsigned>(m);
+  if (k <= kActRegMaxK) {
+    const int threads = slots <= 128 ? ((slots + 31) / 32) * 32 : 128;
+    const int j = (slots + threads - 1) / threads;
+    const int kk = static_cast<int>(k);
+    switch (j) {
+      case 1: act_quant_reg_kernel<1><<<grid, threads, 0, stream>>>(x, kk, rotate, xq, xs); break;
+      case 2: act_quant_reg_kernel<2><<<grid, threads, 0, stream>>>(x, kk, rotate, xq, xs); break;
+      case 3: act_quant_reg_kernel<3><<<grid, threads, 0, stream>>>(x, kk, rotate, xq, xs); break;
+      case 4: act_quant_reg_kernel<4><<<grid, threads, 0, stream>>>(x, kk, rotate, xq, xs); break;
+      case 5: act_quant_reg_kernel<5><<<grid, threads, 0, stream>>>(x, kk, rotate, xq, xs); break;
+      case 6: act_quant_reg_kernel<6><<<grid, threads, 0, stream>>>(x, kk, rotate, xq, xs); break;
+      case 7: act_quant_reg_kernel<7><<<grid, threads, 0, stream>>>(x, kk, rotate, xq, xs); break;
+      default: act_quant_reg_kernel<8><<<grid, threads, 0, stream>>>(x, kk, rotate, xq, xs); break;
+    }
+  } else {
+    act_quant_2pass_kernel<<<grid, kActTwoPassThreads, 0, stream>>>(x, static_cast<int>(k), rotate, xq, xs);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gemv(const LinearArgs& a, cudaStream_t stream) {
+  if (a.m == 0 || a.n == 0) return cudaSuccess;
+  DeviceInfo d;
+  cudaError_t e = device_info(&d);
+  if (e != cudaSuccess) return e;
+  const int step = gemv_max_mt(a.k, d);
+  if (step == 0) return cudaErrorInvalidConfiguration;
+  const int64_t ng = a.k / (a.fmt == 0 ? kGroupTrunk : kGroupHead);
+  for (int64_t m0 = 0; m0 < a.m; m0 += step) {
+    const int mg = static_cast<int>(std::min<int64_t>(step, a.m - m0));
+    LinearArgs s = a;
+    s.m = mg;
+    s.xq = a.xq + m0 * a.k;
+    if (a.xs) s.xs = a.xs + m0;
+    if (a.y) s.y = a.y + m0 * a.n;
+    if (a.partials) s.partials = a.partials + m0 * a.n * ng;
+    const int mt = next_pow2(mg);
+    const bool part = a.partials != nullptr;
+    if (a.fmt == 0)
+      e = part ? launch_gemv_mt<0, true>(s, mt, d, stream) : launch_gemv_mt<0, false>(s, mt, d, stream);
+    else
+      e = part ? launch_gemv_mt<1, true>(s, mt, d, stream) : launch_gemv_mt<1, false>(s, mt, d, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+bool gemv_supported(int64_t k, std::string* why) {
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) {
+    if (why) *why = "cannot query the current device";
+    return false;
+  }
+  if (gemv_max_mt(k, d) == 0) {
+    if (why) *why = "K too large for the GEMV's shared-memory activation buffer";
+    return false;
+  }
+  return true;
+}
+
+bool gemm_tc_supported(const LinearArgs&, std::string* why) {
+  if (why) *why = "the tensor-core path is not available in this build";
+  return false;
+}
+
+cudaError_t launch_gemm_tc(const LinearArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+
+namespace {
+
+// One thread waits on a barrier that nothing will ever arrive on; the
+// bounded wait must give up after limit_ns and record the self-test code.
+__global__ void wait_selftest_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    mbar_wait(&bar, 0u, kDevErrSelftest, limit_ns);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream) {
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);
+  return cudaGetLastError();
+}
+
+cudaError_t read_and_clear_device_error(uint32_t* err) {
+  uint32_t v = 0;
+  cudaError_t e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof(v));
+  if (e != cudaSuccess) return e;
+  if (v != 0) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return e;
+  }
+  *err = v;
+  return cudaSuccess;
+}
+
+}  // namespace iq8r

@@ -1,0 +1,140 @@
+// Host-side round-to-nearest packing of bf16 weights into the IQ8R formats.
+//
+// Trunk ("Qwen3.8-27B IQ8R + DFlash2 -- radiance container", table row
+// "Weights", and the recipe rule "codes=i8 group=256 scale=u8 scale2=bf16
+// block2=1x* transform=fwht128 clamp=sym"): int8 codes -127..127, a u8
+// sub-scale per (row, 256 of K) under a bf16 scale per row, each 128 of K
+// rotated by the unnormalised Hadamard first.
+// lm_head (same row; recipe "codes=i8 group=128 scale=bf16 clamp=sym"): a
+// bf16 scale per (row, 128 of K).
+//
+// The pages fit the codes by GPTQ against calibration Hessians; packing here
+// is the recipes' "rtn" rule with these stated scale definitions:
+//   trunk:   s2 = bf16 of R / (127 * 255) rounded up, R the row's absmax;
+//            s1 = min(255, ceil(A / (127 * s2))), A the 256-block's absmax;
+//            code = clamp(rint(w' / (s2 * s1)), -127, 127).
+//   lm_head: s = bf16 of A / 127 rounded up (A over the 128-block);
+//            code = clamp(rint(w' / s), -127, 127).
+// Every step is one IEEE float32 operation (this file must be compiled
+// without fast-math or FMA contraction), so the bytes are reproducible.
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <thread>
+#include <vector>
+
+#include "iq8r_internal.h"
+
+namespace iq8r {
+namespace {
+
+inline float bf16_to_float(uint16_t b) {
+  uint32_t u = static_cast<uint32_t>(b) << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+inline uint32_t float_bits(float f) {
+  uint32_t u;
+  std::memcpy(&u, &f, 4);
+  return u;
+}
+
+inline float bits_float(uint32_t u) {
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+
+// Smallest bf16 >= v for finite v >= 0: keep the upper 16 bits and step one
+// bf16 unit up if anything was cut off (the same rule covers subnormals).
+inline uint16_t bf16_round_up_bits(float v) {
+  uint32_t u = float_bits(v);
+  uint32_t hi = u & 0xFFFF0000u;
+  if (u & 0x0000FFFFu) hi += 0x00010000u;
+  return static_cast<uint16_t>(hi >> 16);
+}
+
+// In-place fwht128 on 128 floats: stages h = 1, 2, 4, ..., 64 in that order,
+// (a, b) -> (a + b, a - b).
+inline void fwht128(float* v) {
+  for (int h = 1; h < kRot; h <<= 1) {
+    for (int i = 0; i < kRot; i += 2 * h) {
+      for (int j = i; j < i + h; ++j) {
+        const float a = v[j];
+        const float b = v[j + h];
+        v[j] = a + b;
+        v[j + h] = a - b;
+      }
+    }
+  }
+}
+
+inline int8_t quantise(float w, float step) {
+  if (!(step > 0.0f)) return 0;
+  float q = std::nearbyint(w / step);  // round-half-even (default mode)
+  q = std::min(127.0f, std::max(-127.0f, q));
+  return static_cast<int8_t>(q);
+}
+
+void pack_range(int fmt, bool rotate, const uint16_t* w, int64_t k, int64_t r0, int64_t r1,
+                int8_t* codes, uint8_t* sub, uint16_t* scale) {
+  std::vector<float> row(static_cast<size_t>(k));
+  const int64_t g256 = k / kGroupTrunk;
+  const int64_t g128 = k / kGroupHead;
+  std::vector<float> amax(static_cast<size_t>(std::max<int64_t>(g128, 1)));
+  for (int64_t r = r0; r < r1; ++r) {
+    const uint16_t* src = w + r * k;
+    for (int64_t i = 0; i < k; ++i) row[i] = bf16_to_float(src[i]);
+    if (rotate)
+      for (int64_t c = 0; c < k; c += kRot) fwht128(row.data() + c);
+    int8_t* out = codes + r * k;
+    if (fmt == 0) {
+      float R = 0.0f;
+      for (int64_t g = 0; g < g256; ++g) {
+        float A = 0.0f;
+        for (int64_t i = g * kGroupTrunk; i < (g + 1) * kGroupTrunk; ++i) A = std::max(A, std::fabs(row[i]));
+        amax[g] = A;
+        R = std::max(R, A);
+      }
+      const uint16_t s2b = bf16_round_up_bits(R / 32385.0f);
+      const float s2 = bf16_to_float(s2b);
+      scale[r] = s2b;
+      const float den = 127.0f * s2;  // exact: 7-bit x 8-bit significands
+      for (int64_t g = 0; g < g256; ++g) {
+        float s1 = 0.0f;
+        if (s2 > 0.0f) s1 = std::min(255.0f, std::ceil(amax[g] / den));
+        sub[r * g256 + g] = static_cast<uint8_t>(s1);
+        const float d = s2 * s1;  // exact: 8-bit x 8-bit significands
+        for (int64_t i = g * kGroupTrunk; i < (g + 1) * kGroupTrunk; ++i) out[i] = quantise(row[i], d);
+      }
+    } else {
+      for (int64_t g = 0; g < g128; ++g) {
+        float A = 0.0f;
+        for (int64_t i = g * kGroupHead; i < (g + 1) * kGroupHead; ++i) A = std::max(A, std::fabs(row[i]));
+        const uint16_t sb = bf16_round_up_bits(A / 127.0f);
+        scale[r * g128 + g] = sb;
+        const float s = bf16_to_float(sb);
+        for (int64_t i = g * kGroupHead; i < (g + 1) * kGroupHead; ++i) out[i] = quantise(row[i], s);
+      }
+    }
+  }
+}
+
+}  // namespace
+
+void pack_rows(int fmt, bool rotate, const uint16_t* w, int64_t n, int64_t k, int8_t* codes,
+               uint8_t* sub, uint16_t* scale, int n_threads) {
+  if (n_threads <= 0) n_threads = static_cast<int>(std::max(1u, std::thread::hardware_concurrency()));
+  const int64_t per = std::max<int64_t>(64, (n + n_threads - 1) / n_threads);
+  std::vector<std::thread> pool;
+  for (int64_t r0 = 0; r0 < n; r0 += per) {
+    const int64_t r1 = std::min(n, r0 + per);
+    pool.emplace_back(pack_range, fmt, rotate, w, k, r0, r1, codes, sub, scale);
+  }
+  for (auto& t : pool) t.join();
+}
+
+}  // namespace iq8r

@@ -1,0 +1,265 @@
+"""CUDA path against the oracle, through the C ABI (needs a B200).
+
+Bit-exact: activation codes and scales, per-block int32 partial sums.
+Within tolerance (see tolerance.py): the bf16 outputs.
+"""
+
+import functools
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantised_fwht128_act_b200 as iq8r
+from iq8r_inputs import f32_to_bf16_bits, gen_workload
+from tolerance import check_output
+
+pytestmark = pytest.mark.gpu
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def host_bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from quantised_fwht128_act_b200 import build
+    build.build()
+    iq8r.lib()
+    yield
+    iq8r.iq8r_get_device_error()
+
+
+@functools.lru_cache(maxsize=8)
+def case(name, m=None, n=None, k=None, seed=None):
+    """Inputs, oracle-packed weight and device copies for one configuration."""
+    x, w = gen_workload(name, m=m, n=n, k=k, seed=seed)
+    fmt = "g128" if name.startswith("lm_head") else "g256"
+    codes, sub, scale = oracle.pack(w, fmt, True)
+    W = iq8r.IQ8RWeight.from_packed(codes, sub, scale, fmt, True)
+    return x, w, fmt, (codes, sub, scale), W
+
+
+def run_act(x_bits, rotate=True):
+    xq, xs = iq8r.iq8r_rotate_quant_act(dev_bf16(x_bits), rotate)
+    torch.cuda.synchronize()
+    return xq.cpu().numpy(), xs.cpu().numpy()
+
+
+def assert_act_exact(x_bits, rotate=True):
+    q0, a0 = oracle.act_quant(x_bits, rotate)
+    q1, a1 = run_act(x_bits, rotate)
+    assert np.array_equal(q0, q1), f"{np.sum(q0 != q1)} codes differ"
+    assert np.array_equal(a0.view(np.uint32), a1.view(np.uint32))
+
+
+# ------------------------------------------------------------ activations
+
+@pytest.mark.parametrize("name", ["pr1", "decode", "verify8", "verify128", "lm_head8"])
+def test_act_bit_exact_workloads(name):
+    x, _ = gen_workload(name, n=8)
+    assert_act_exact(x)
+
+
+def test_act_bit_exact_prefill_full():
+    x, _ = gen_workload("prefill", n=8)
+    assert_act_exact(x)
+
+
+@pytest.mark.parametrize("m,k", [(5, 128), (3, 640), (7, 2176), (1, 16384), (2, 16512), (3, 33024), (33, 1152)])
+def test_act_bit_exact_ragged_shapes(m, k):
+    x, _ = gen_workload("decode", m=m, n=8, k=k, seed=m * 1000 + k)
+    assert_act_exact(x)
+    assert_act_exact(x, rotate=False)
+
+
+def test_act_special_rows():
+    k = 1024
+    rng = np.random.default_rng(3)
+    x = np.zeros((6, k), np.float32)
+    x[1, 700] = -3.25                                   # spike
+    x[2] = rng.standard_normal(k) * 1e37                # near the top of the range
+    x[3] = rng.standard_normal(k) * 1e-39               # bf16 subnormals
+    x[4] = np.round(rng.standard_normal(k) * 4)         # exact small integers
+    x[5] = rng.standard_normal(k) * np.exp(rng.uniform(-30, 30, k))
+    bits = f32_to_bf16_bits(x)
+    assert_act_exact(bits)
+    assert_act_exact(bits, rotate=False)
+
+
+def test_act_empty_batch_is_a_no_op():
+    x = torch.zeros((0, 256), dtype=torch.bfloat16, device="cuda")
+    xq, xs = iq8r.iq8r_rotate_quant_act(x)
+    assert xq.shape == (0, 256) and xs.shape == (0,)
+
+
+# ------------------------------------------------------------- partials
+
+def gpu_partials(x_bits, W, n0=0, n1=None, path=iq8r.IQ8R_PATH_AUTO):
+    xq, _ = iq8r.iq8r_rotate_quant_act(dev_bf16(x_bits))
+    p = iq8r.iq8r_linear_partials(xq, W, n0, n1, path=path)
+    torch.cuda.synchronize()
+    return p.cpu().numpy()
+
+
+@pytest.mark.parametrize("name", ["pr1", "decode", "verify8"])
+def test_partials_bit_exact_workloads(name):
+    x, _, fmt, (codes, _, _), W = case(name)
+    g = 256 if fmt == "g256" else 128
+    xq, _ = oracle.act_quant(x)
+    assert np.array_equal(gpu_partials(x, W), oracle.partials(xq, codes, g))
+
+
+@pytest.mark.parametrize("m,n,k", [(3, 1000, 768), (5, 37, 2304), (13, 64, 512), (2, 9, 4352), (8, 20, 256)])
+def test_partials_bit_exact_ragged(m, n, k):
+    x, _, _, (codes, _, _), W = case("decode", m=m, n=n, k=k, seed=7 + m + n + k)
+    xq, _ = oracle.act_quant(x)
+    assert np.array_equal(gpu_partials(x, W), oracle.partials(xq, codes, 256))
+
+
+def test_partials_lm_head_windows():
+    x, _, _, (codes, _, _), W = case("lm_head8", m=8, n=4096, k=5120, seed=44)
+    xq, _ = oracle.act_quant(x)
+    for n0, n1 in [(0, 8), (8, 1000), (4090, 4096), (1234, 2345)]:
+        got = gpu_partials(x, W, n0, n1)
+        assert np.array_equal(got, oracle.partials(xq, codes[n0:n1], 128))
+
+
+def test_partials_extreme_codes():
+    # |P| reaches 256 * 127^2 = 4129024 when every code is +-127
+    k, n = 512, 16
+    x = np.zeros((2, k), np.float32)
+    x[0, 0] = 1.0       # rotates to +-1 over the chunk -> codes +-127
+    x[1, 128] = -2.0
+    xb = f32_to_bf16_bits(x)
+    codes = np.full((n, k), 127, np.int8)
+    codes[1::2] = -127
+    sub = np.full((n, k // 256), 255, np.uint8)
+    scale = np.full((n,), 0x3C00, np.uint16)
+    W = iq8r.IQ8RWeight.from_packed(codes, sub, scale, "g256", True)
+    xq, _ = oracle.act_quant(xb)
+    assert np.array_equal(gpu_partials(xb, W), oracle.partials(xq, codes, 256))
+
+
+# ---------------------------------------------------------------- linear
+
+def gpu_linear(x_bits, W, path=iq8r.IQ8R_PATH_AUTO):
+    xq, xs = iq8r.iq8r_rotate_quant_act(dev_bf16(x_bits))
+    y = iq8r.iq8r_linear_ex(xq, xs, W, path=path)
+    torch.cuda.synchronize()
+    return host_bits(y)
+
+
+def oracle_linear(x, fmt, packed):
+    codes, sub, scale = packed
+    xq, a = oracle.act_quant(x)
+    return oracle.linear(xq, a, fmt, codes, sub, scale, rotated=True)
+
+
+@pytest.mark.parametrize("name", ["pr1", "decode", "verify8", "verify16", "verify128"])
+def test_linear_within_tolerance_workloads(name):
+    x, _, fmt, packed, W = case(name)
+    y64 = oracle_linear(x, fmt, packed)
+    st = check_output(gpu_linear(x, W), y64, oracle.linear_bf16(y64))
+    assert st["bit_equal_frac"] > 0.99
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 1000, 768), (3, 37, 2304), (13, 64, 512), (5, 9, 4352), (2, 333, 1280)])
+def test_linear_within_tolerance_ragged(m, n, k):
+    x, _, fmt, packed, W = case("decode", m=m, n=n, k=k, seed=11 + m + n + k)
+    y64 = oracle_linear(x, fmt, packed)
+    check_output(gpu_linear(x, W), y64, oracle.linear_bf16(y64))
+
+
+def test_linear_lm_head_small():
+    x, _, fmt, packed, W = case("lm_head8", m=8, n=2000, k=5120, seed=45)
+    y64 = oracle_linear(x, fmt, packed)
+    check_output(gpu_linear(x, W), y64, oracle.linear_bf16(y64))
+
+
+def test_linear_unrotated_weight():
+    x, w = gen_workload("pr1")
+    codes, sub, scale = oracle.pack(w, "g256", rotate=False)
+    W = iq8r.IQ8RWeight.from_packed(codes, sub, scale, "g256", rotated=False)
+    xq, xs = iq8r.iq8r_rotate_quant_act(dev_bf16(x), rotate=False)
+    y = host_bits(iq8r.iq8r_linear(xq, xs, W))
+    q, a = oracle.act_quant(x, rotate=False)
+    y64 = oracle.linear(q, a, "g256", codes, sub, scale, rotated=False)
+    check_output(y, y64)
+
+
+def test_linear_zero_activation_row_gives_zero():
+    x, _, fmt, packed, W = case("pr1")
+    x = x.copy()
+    x[2] = 0
+    y = gpu_linear(x, W)
+    assert np.all(y[2] == 0)
+
+
+def test_prefill_full_size_sampled_rows():
+    """M = 8192 through the library's launch configuration; the oracle checks
+    a sample of token rows (all N outputs of each) and every act code."""
+    x, _, fmt, packed, W = case("prefill")
+    xq_d, xs_d = iq8r.iq8r_rotate_quant_act(dev_bf16(x))
+    y = host_bits(iq8r.iq8r_linear(xq_d, xs_d, W))
+    q, a = oracle.act_quant(x)
+    assert np.array_equal(q, xq_d.cpu().numpy())
+    rows = np.random.default_rng(0).choice(x.shape[0], 24, replace=False)
+    rows = np.concatenate([rows, [0, x.shape[0] - 1]])
+    codes, sub, scale = packed
+    y64 = oracle.linear(q[rows], a[rows], fmt, codes, sub, scale, rotated=True)
+    check_output(y[rows], y64)
+    assert np.array_equal(gpu_partials(x[rows], W, 0, 17408),
+                          oracle.partials(q[rows], codes, 256))
+
+
+def test_lm_head_full_top32():
+    """Full lm_head (N = 151936): outputs within tolerance, and the top-32
+    logits agree with the oracle's: every oracle top-32 entry is within the
+    output tolerance of the GPU's 32nd value and vice versa (the order of
+    near-equal logits is not unique after bf16 rounding)."""
+    _, w = gen_workload("lm_head8")           # the weight is drawn first: same for M = 1 and 8
+    codes, sub, scale = oracle.pack(w, "g128", True)
+    del w
+    W = iq8r.IQ8RWeight.from_packed(codes, sub, scale, "g128", True)
+    for name in ("lm_head1", "lm_head8"):
+        x, _ = gen_workload(name, n=8)
+        y = gpu_linear(x, W)
+        y64 = oracle_linear(x, "g128", (codes, sub, scale))
+        check_output(y, y64)
+        yg = (y.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+        tol = 1e-2 * np.sqrt(np.mean(y64 ** 2))
+        for i in range(x.shape[0]):
+            top_ref = np.argsort(-y64[i], kind="stable")[:32]
+            top_gpu = np.argsort(-yg[i], kind="stable")[:32]
+            thr_ref = y64[i, top_ref[-1]]
+            thr_gpu = yg[i, top_gpu[-1]]
+            ulp = 2.0 ** (np.floor(np.log2(abs(thr_gpu))) - 7)
+            assert np.all(yg[i, top_ref] >= thr_gpu - tol - ulp)
+            assert np.all(y64[i, top_gpu] >= thr_ref - tol - ulp)
+            assert len(set(top_ref) & set(top_gpu)) >= 30
+    del W
+    torch.cuda.empty_cache()
+
+
+def test_device_error_word_is_clear_after_the_suite_so_far():
+    iq8r.iq8r_get_device_error()
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    iq8r.iq8r_get_device_error()
+    iq8r.iq8r_selftest_wait_timeout(2_000_000)
+    with pytest.raises(iq8r.IQ8RError) as e:
+        iq8r.iq8r_get_device_error()
+    assert e.value.status == iq8r.IQ8R_ERR_DEVICE_TIMEOUT
+    assert "self-test" in str(e.value)
+    iq8r.iq8r_get_device_error()  # cleared
+    # the context still works
+    x, _, fmt, packed, W = case("pr1")
+    y64 = oracle_linear(x, fmt, packed)
+    check_output(gpu_linear(x, W), y64)
