@@ -42,10 +42,11 @@ cudaError_t device_info(DeviceInfo* out) {
 }
 
 // Raise a kernel's dynamic shared memory limit once per device (and again
-// only if a larger size is asked for).
+// only if a larger size is asked for). `configured` must be distinct for
+// every kernel: kernels of one signature share a function-pointer type, so
+// the caller owns the cache (a static inside its own template instance).
 template <typename Kernel>
-cudaError_t ensure_smem(Kernel kernel, int bytes) {
-  static std::atomic<int> configured[kMaxDevices];
+cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<int>* configured) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -63,13 +64,14 @@ template <int MT, int FMT, bool PARTIALS>
 cudaError_t launch_gemv_t(const LinearArgs& a, const DeviceInfo& d, cudaStream_t stream) {
   const int k = static_cast<int>(a.k);
   const int red = gemv_red_bytes<MT, FMT>();
-  const int base = gemv_smem_bytes(MT, k, 0, red);
   const int budget = d.smem_optin - kSmemReserve;
-  const int stages = std::min(kGemvMaxStages, (budget - base) / (kGemvStageBytes + 16));
+  int stages = kGemvMaxStages;
+  while (stages >= 2 && gemv_smem_layout(MT, FMT, k, stages, red).total > budget) --stages;
   if (stages < 2) return cudaErrorInvalidConfiguration;
-  const int smem = gemv_smem_bytes(MT, k, stages, red);
+  const int smem = gemv_smem_layout(MT, FMT, k, stages, red).total;
   auto kernel = gemv_kernel<MT, FMT, PARTIALS>;
-  cudaError_t e = ensure_smem(kernel, smem);
+  static std::atomic<int> configured[kMaxDevices];
+  cudaError_t e = ensure_smem(kernel, smem, configured);
   if (e != cudaSuccess) return e;
   const int64_t tiles = (a.n + kGemvRows - 1) / kGemvRows;
   const int64_t grid = std::min<int64_t>(d.num_sms, tiles);
@@ -96,8 +98,9 @@ int next_pow2(int v) {
 // Largest token tile (1, 2, 4 or 8) whose activation codes leave room for a
 // two-stage ring.
 int gemv_max_mt(int64_t k, const DeviceInfo& d) {
+  if (k > (int64_t(1) << 24)) return 0;
   for (int mt = 8; mt >= 1; mt >>= 1) {
-    const int need = gemv_smem_bytes(mt, static_cast<int>(k), 2, 2 * 8 * 8 * 8);
+    const int need = gemv_smem_layout(mt, 1, static_cast<int>(k), 2, 2 * 8 * 8 * 8).total;
     if (need <= d.smem_optin - kSmemReserve) return mt;
   }
   return 0;

@@ -83,7 +83,7 @@ def test_act_special_rows():
     rng = np.random.default_rng(3)
     x = np.zeros((6, k), np.float32)
     x[1, 700] = -3.25                                   # spike
-    x[2] = rng.standard_normal(k) * 1e37                # near the top of the range
+    x[2] = rng.standard_normal(k) * 1e35                # large, transform stays finite
     x[3] = rng.standard_normal(k) * 1e-39               # bf16 subnormals
     x[4] = np.round(rng.standard_normal(k) * 4)         # exact small integers
     x[5] = rng.standard_normal(k) * np.exp(rng.uniform(-30, 30, k))
