@@ -72,7 +72,16 @@ def linear_bytes(m, k, n, fmt):
     return w + m * k + 4 * m + 2 * m * n
 
 
+def fused_bytes(m, k, n, fmt):
+    """One-launch layer: bf16 activations in, weights, bf16 out."""
+    return linear_bytes(m, k, n, fmt) - m * k - 4 * m + 2 * m * k
+
+
 def step_bytes(m, k, n, fmt):
+    """Algorithmic bytes of one step: the fused layer for M <= 8, else the
+    activation kernel plus the linear."""
+    if m <= 8:
+        return fused_bytes(m, k, n, fmt)
     return act_bytes(m, k) + linear_bytes(m, k, n, fmt)
 
 
@@ -217,12 +226,16 @@ def run_ours(args, rank, world, local_rank):
     xq = [torch.empty((m, k), dtype=torch.int8, device=dev) for _ in range(R)]
     xsc = [torch.empty((m,), dtype=torch.float32, device=dev) for _ in range(R)]
     y = [torch.empty((m, n), dtype=torch.bfloat16, device=dev) for _ in range(R)]
-    launches_per_step = 2 + (0 if m <= 8 else (m + 7) // 8 - 1)  # act + GEMV groups of 8 tokens
+    fused = m <= 8  # one launch: the GEMV rotates and quantises x itself
+    launches_per_step = 1 if fused else 1 + (m + 7) // 8  # else act + GEMV groups of 8 tokens
 
     def step(j):
         r = j % R
-        iq8r.iq8r_rotate_quant_act(x_dev[r], True, xq[r], xsc[r])
-        iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
+        if fused:
+            iq8r.iq8r_linear_bf16(x_dev[r], weights[r], y[r])
+        else:
+            iq8r.iq8r_rotate_quant_act(x_dev[r], True, xq[r], xsc[r])
+            iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
@@ -244,9 +257,13 @@ def run_ours(args, rank, world, local_rank):
             for j in range(nsteps):
                 r = (offset + j) % R
                 evs[j][0].record()
-                iq8r.iq8r_rotate_quant_act(x_dev[r], True, xq[r], xsc[r])
+                if not fused:
+                    iq8r.iq8r_rotate_quant_act(x_dev[r], True, xq[r], xsc[r])
                 evs[j][1].record()
-                iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
+                if fused:
+                    iq8r.iq8r_linear_bf16(x_dev[r], weights[r], y[r])
+                else:
+                    iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
                 evs[j][2].record()
         return g, evs
 
@@ -306,8 +323,11 @@ def run_ours(args, rank, world, local_rank):
             for j in range(min(W, 50)):
                 r = j % R
                 xin[r].copy_(xh[r], non_blocking=True)
-                iq8r.iq8r_rotate_quant_act(xin[r], True, xq[r], xsc[r])
-                iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
+                if fused:
+                    iq8r.iq8r_linear_bf16(xin[r], weights[r], y[r])
+                else:
+                    iq8r.iq8r_rotate_quant_act(xin[r], True, xq[r], xsc[r])
+                    iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
                 yh[r].copy_(y[r], non_blocking=True)
         stream.synchronize()
         if world > 1:
@@ -320,8 +340,11 @@ def run_ours(args, rank, world, local_rank):
             for j in range(Ke):
                 r = j % R
                 xin[r].copy_(xh[r], non_blocking=True)
-                iq8r.iq8r_rotate_quant_act(xin[r], True, xq[r], xsc[r])
-                iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
+                if fused:
+                    iq8r.iq8r_linear_bf16(xin[r], weights[r], y[r])
+                else:
+                    iq8r.iq8r_rotate_quant_act(xin[r], True, xq[r], xsc[r])
+                    iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
                 yh[r].copy_(y[r], non_blocking=True)
             s1.record()
         stream.synchronize()
@@ -337,11 +360,12 @@ def run_ours(args, rank, world, local_rank):
     hbm, bf16_tf, peak_src = peaks()
     lin_avg_ms = float(np.mean(lin_ms))
     act_avg_ms = float(np.mean(act_ms))
-    lin_b = linear_bytes(m, k, n, fmt)
-    kern_files = ["gemv.cuh", "iq8r_device.cuh"]
+    lin_b = fused_bytes(m, k, n, fmt) if fused else linear_bytes(m, k, n, fmt)
+    kern_files = ["gemv.cuh", "act_quant.cuh", "iq8r_device.cuh"]
     if m <= 8:
         achieved = lin_b / (lin_avg_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "kernel": "gemv_kernel", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+        roof = {"bound": "hbm", "kernel": "gemv_kernel (fused act, one launch per step)", "achieved": achieved,
+                "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "peak_source": f"{peak_src} HBM copy (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_src == "measured" else "fallback 6.65 TB/s",
                 "traffic": recorded_traffic("gemv_kernel", args.config, kern_files),
@@ -354,8 +378,9 @@ def run_ours(args, rank, world, local_rank):
                 "int8_tops": ops / (lin_avg_ms * 1e-3) / 1e12,
                 "traffic": recorded_traffic("gemv_kernel", args.config, kern_files),
                 "algorithmic_bytes_per_launch": lin_b, "avg_launch_ms": lin_avg_ms}
-    roof["act_kernel"] = {"avg_launch_ms": act_avg_ms, "bytes": act_bytes(m, k),
-                          "achieved_gbs": act_bytes(m, k) / (act_avg_ms * 1e-3) / 1e9}
+    if not fused:
+        roof["act_kernel"] = {"avg_launch_ms": act_avg_ms, "bytes": act_bytes(m, k),
+                              "achieved_gbs": act_bytes(m, k) / (act_avg_ms * 1e-3) / 1e9}
 
     value = world * step_bytes(m, k, n, fmt) * K / (elapsed_ms * 1e-3) / 1e9
     clocks = sampler.summary(t_start_wall, t_end_wall)
@@ -364,7 +389,7 @@ def run_ours(args, rank, world, local_rank):
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8", "data": "synthetic",
         "config": {"workload": args.config, "m": m, "k": k, "n": n, "format": fmt, "rotated": True,
-                   "step": "iq8r_rotate_quant_act + iq8r_linear",
+                   "step": "iq8r_linear_bf16 (one launch)" if fused else "iq8r_rotate_quant_act + iq8r_linear",
                    "bytes_per_step": step_bytes(m, k, n, fmt),
                    "l2": f"{R} rotating weight/input copies ({R * footprint / 1e6:.0f} MB > 3x L2)" if R > 1
                    else "a step moves more than 3x L2",

@@ -81,8 +81,8 @@ typedef enum {
  *   scale     bf16 [n] (G256) or [n][k/128] (G128), as raw 16-bit patterns
  *   rotated   1 if the codes live in the fwht128 domain (the output is then
  *             multiplied by 1/128); 0 for a plain int8 weight.
- * k must be a multiple of 256 (G256) or 128 (G128); codes and scale must be
- * 16-byte aligned; sub_scale needs no alignment. */
+ * k must be a multiple of 256 (G256) or 128 (G128); codes, sub_scale and
+ * scale must be 16-byte aligned (the arrays' base addresses). */
 typedef struct {
   int32_t fmt;
   int32_t rotated;
@@ -138,6 +138,22 @@ iq8r_status iq8r_rotate_quant_act(const uint16_t* x_bf16, int64_t m, int64_t k, 
  * rounding plus ~1e-6 of the output's scale. */
 iq8r_status iq8r_linear(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,
                         uint16_t* y_bf16, cudaStream_t stream);
+
+/* The whole layer from bf16 activations: rotate + quantise x (as
+ * iq8r_rotate_quant_act, rotating iff w->rotated) and then iq8r_linear.
+ * For m <= 8 and m * k <= 16384 (a decode step), or when xq_out and
+ * x_scale_out are not given, this is one kernel: every CTA of the
+ * weight-streaming GEMV rotates and quantises x itself while its first
+ * weight tiles stream in. Otherwise the codes are staged in xq_out /
+ * x_scale_out and a second kernel consumes them.
+ *   x_bf16      device bf16 [m][w->k], 16-byte aligned (w->k % 128 == 0)
+ *   y_bf16      device bf16 [m][w->n] (out), 16-byte aligned
+ *   xq_out      device int8 [m][w->k] (out) or NULL: the activation codes
+ *   x_scale_out device fp32 [m] (out) or NULL: the activation scales
+ * For m > 8 xq_out / x_scale_out must be given. Codes and y are the same
+ * bits either way, and the same as the two-call path. */
+iq8r_status iq8r_linear_bf16(const uint16_t* x_bf16, int64_t m, const iq8r_weight* w, uint16_t* y_bf16,
+                             int8_t* xq_out, float* x_scale_out, cudaStream_t stream);
 
 /* iq8r_linear with an explicit kernel choice (tests and measurement). */
 iq8r_status iq8r_linear_ex(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,

@@ -24,7 +24,7 @@ __all__ = [
     "IQ8R_FMT_G256_U8_BF16", "IQ8R_FMT_G128_BF16", "IQ8R_PATH_AUTO", "IQ8R_PATH_GEMV", "IQ8R_PATH_TC",
     "IQ8RError", "IQ8RWeight", "lib", "lib_path",
     "iq8r_version", "iq8r_last_error", "iq8r_packed_sizes", "iq8r_pack", "iq8r_rotate_quant_act",
-    "iq8r_linear", "iq8r_linear_ex", "iq8r_linear_partials", "iq8r_get_device_error",
+    "iq8r_linear", "iq8r_linear_bf16", "iq8r_linear_ex", "iq8r_linear_partials", "iq8r_get_device_error",
     "iq8r_selftest_wait_timeout",
 ]
 
@@ -91,6 +91,8 @@ def lib():
     L.iq8r_rotate_quant_act.argtypes = [vp, i64, i64, i32, vp, vp, vp]
     L.iq8r_linear.restype = i32
     L.iq8r_linear.argtypes = [vp, vp, i64, ctypes.POINTER(_Weight), vp, vp]
+    L.iq8r_linear_bf16.restype = i32
+    L.iq8r_linear_bf16.argtypes = [vp, i64, ctypes.POINTER(_Weight), vp, vp, vp, vp]
     L.iq8r_linear_ex.restype = i32
     L.iq8r_linear_ex.argtypes = [vp, vp, i64, ctypes.POINTER(_Weight), vp, i32, vp]
     L.iq8r_linear_partials.restype = i32
@@ -232,6 +234,27 @@ def iq8r_linear(xq, x_scale, weight: IQ8RWeight, y=None, stream=None):
         y = torch.empty((m, weight.n), dtype=torch.bfloat16, device=xq.device)
     w = weight._struct()
     _check(lib().iq8r_linear(_ptr(xq), _ptr(x_scale), m, ctypes.byref(w), _ptr(y), _stream(stream)))
+    return y
+
+
+def iq8r_linear_bf16(x, weight: IQ8RWeight, y=None, xq_out=None, x_scale_out=None, stream=None):
+    """y = x W^T from bf16 activations [M, K] (rotated and quantised inside;
+    one launch for M <= 8). xq_out / x_scale_out receive the activation codes
+    and scales when given (required for M > 8)."""
+    import torch
+    if x.dim() != 2 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous [M, K] tensor")
+    m = x.shape[0]
+    if y is None:
+        y = torch.empty((m, weight.n), dtype=torch.bfloat16, device=x.device)
+    if m > 8:
+        if xq_out is None:
+            xq_out = torch.empty((m, weight.k), dtype=torch.int8, device=x.device)
+        if x_scale_out is None:
+            x_scale_out = torch.empty((m,), dtype=torch.float32, device=x.device)
+    w = weight._struct()
+    _check(lib().iq8r_linear_bf16(_ptr(x), m, ctypes.byref(w), _ptr(y), _ptr(xq_out), _ptr(x_scale_out),
+                                  _stream(stream)))
     return y
 
 

@@ -8,75 +8,96 @@
 // page's "Speed" section: the IQ8R decode step runs as fast as FP8's, the
 // same bytes a weight).
 //
-// Design (sm_100a):
-//  - persistent grid, one CTA per SM, each CTA a contiguous range of 8-row
-//    tiles (balanced to one tile);
-//  - warp 8 is the producer. One lane issues every copy with 1-D bulk copies
-//    (TMA engine) completing on mbarriers: the activation codes once, then
-//    per tile its scales (u8 sub-scales and bf16 row scales, or the lm_head's
-//    bf16 group scales) into a 4-slot scale ring, and the tile's codes in
-//    2 KB-of-K chunks (8 rows x 2 KB = 16 KB stage) into a ring of up to 12
-//    stages, weights marked evict-first in L2;
-//  - warps 0..7 consume from shared memory only: a warp owns RG rows and
-//    every WK-th 512-byte step of K; each lane does 4 dp4a per 16 bytes per
-//    token, scales the lane's partial by its block's u8 sub-scale in int32
-//    (exact) and folds it into int64 once per chunk;
-//  - epilogue: warp shuffle (and, when WK > 1, a shared-memory) reduction,
-//    then the fp32 scale product and one bf16 rounding.
+// Design (sm_100a), warp-autonomous streaming:
+//  - persistent grid, one CTA per SM, each CTA a contiguous range of tiles
+//    (balanced to one tile). A tile is RT whole weight rows (contiguous in
+//    memory), or, when a row is longer than a stage, one row in K chunks;
+//  - no producer warp: each of the 8 warps owns D private stage buffers and
+//    keeps them full itself. One lane claims the next tile from a per-CTA
+//    counter and issues 1-D bulk copies (TMA engine) of the stage's codes and
+//    scales (u8 sub-scales + bf16 row scales, or the lm_head's bf16 group
+//    scales) completing on the buffer's mbarrier, weights evict-first in L2.
+//    Only the activation codes are shared, loaded once;
+//  - the warp consumes stages in the order it issued them: per 512-byte step
+//    each lane holds 16 bytes of K; loads for 4 steps are issued before any
+//    dp4a; activation registers are reused across the RG rows computed
+//    together; the lane's partial is scaled by its block's u8 sub-scale in
+//    int32 (exact) and folded into int64 every 16 steps;
+//  - epilogue per tile: warp shuffles, the fp32 scale product and one bf16
+//    rounding per output.
 // PARTIALS instantiates the same loads and dp4a chains but reduces each
 // block's 16 (or 8) lanes and writes P instead of y (the debug twin).
 #pragma once
 
 #include <type_traits>
 
+#include "act_quant.cuh"
 #include "iq8r_device.cuh"
 
 namespace iq8r {
 
-constexpr int kGemvRows = 8;         // rows per tile
-constexpr int kGemvKC = 2048;        // bytes of K per chunk
-constexpr int kGemvStageBytes = kGemvRows * kGemvKC;
-constexpr int kGemvConsumerWarps = 8;
-constexpr int kGemvThreads = (kGemvConsumerWarps + 1) * 32;
-constexpr int kGemvMaxStages = 12;
-constexpr int kGemvScaleSlots = 4;
+constexpr int kGemvMaxWarps = 16;
 
-template <int MT>
-struct GemvShape {
-  static constexpr int RG = MT == 1 ? 1 : (MT == 2 ? 2 : 4);  // rows per warp
-  static constexpr int WR = kGemvRows / RG;                    // warps along rows
-  static constexpr int WK = kGemvConsumerWarps / WR;           // warps along K
-  static constexpr int STEPS = kGemvKC / 512;                  // 512-byte steps per chunk
-  static constexpr int SPW = STEPS / WK;                       // steps per warp per chunk
-};
+// Warps per CTA: more warps hide more load latency; large token tiles need
+// the registers of fewer threads.
+__host__ __device__ constexpr int gemv_warps(int mt) { return mt <= 2 ? 16 : 8; }
+constexpr int kGemvMaxDepth = 4;          // stage buffers per warp
+constexpr int kGemvMaxRowsPerTile = 32;
+constexpr int kGemvMaxCopy = 16 * 1024;   // bytes per bulk copy
+
+// 512-byte steps whose loads are issued together: 4, fewer when the loaded
+// int4 registers (MT activations + RG weights per step) would crowd out the rest.
+__host__ __device__ constexpr int gemv_unroll(int mt, int rg) {
+  return 96 / (4 * (mt + rg)) >= 4 ? 4 : (96 / (4 * (mt + rg)) >= 2 ? 2 : 1);
+}
 
 __host__ __device__ constexpr int gemv_align128(int x) { return (x + 127) & ~127; }
 __host__ __device__ constexpr int gemv_align16(int x) { return (x + 15) & ~15; }
 
-// One tile's scales in shared memory. Trunk: [8][ng] u8 sub-scales, padded
-// to 16 bytes, then [8] bf16 row scales. lm_head: [8][ng] bf16 group scales.
-__host__ __device__ constexpr int gemv_s2_offset(int k) { return gemv_align16(kGemvRows * (k / kGroupTrunk)); }
-__host__ __device__ constexpr int gemv_scale_slot_bytes(int fmt, int k) {
-  return fmt == 0 ? gemv_s2_offset(k) + 2 * kGemvRows : gemv_align16(kGemvRows * (k / kGroupHead) * 2);
-}
-
-template <int MT, int FMT>
-__host__ __device__ constexpr int gemv_red_bytes() {
-  // [2 buffers][WK][WR][RG][MT] of int64 (trunk) or float (lm_head)
-  return 2 * GemvShape<MT>::WK * GemvShape<MT>::WR * GemvShape<MT>::RG * MT * (FMT == 0 ? 8 : 4);
-}
-
-struct GemvSmem {
-  int ring, scales, bars, red, total;
+// Runtime shape of one launch (chosen on the host, see gemv_plan).
+struct GemvPlan {
+  int warps;        // warps per CTA (each streams its own stages)
+  int rt;           // rows per tile
+  int kc;           // bytes of K per stage: K, or a chunk when one row is split
+  int depth;        // stage buffers per warp
+  int stage_bytes;  // codes + scales of one stage, 128-aligned
+  int sc_off;       // offset of the scales within a stage
+  int s2_off;       // offset of the trunk's row scales within a stage
+  int smem;         // total dynamic shared memory
 };
 
-// Shared memory map: [act MT*K][ring][scale slots][barriers][reduction].
-__host__ __device__ constexpr GemvSmem gemv_smem_layout(int mt, int fmt, int k, int stages, int red_bytes) {
-  const int ring = gemv_align128(mt * k);
-  const int scales = ring + stages * kGemvStageBytes;
-  const int bars = scales + kGemvScaleSlots * gemv_scale_slot_bytes(fmt, k);
-  const int red = gemv_align16(bars + 8 * (2 * stages + 2 * kGemvScaleSlots + 1));
-  return GemvSmem{ring, scales, bars, red, red + red_bytes};
+// Scale bytes of one stage: sub-scales (or group scales) for rt rows x kc,
+// then (trunk) rt bf16 row scales. Each is fetched as the 16-byte-aligned
+// window around its bytes, hence up to 32 bytes of slack per array.
+__host__ __device__ constexpr int gemv_s1_window(int rt, int kc) { return gemv_align16(rt * (kc / kGroupTrunk) + 32); }
+__host__ __device__ constexpr int gemv_sc_bytes(int fmt, int rt, int kc) {
+  return fmt == 0 ? gemv_s1_window(rt, kc) + gemv_align16(2 * rt + 32)
+                  : gemv_align16(rt * (kc / kGroupHead) * 2 + 32);
+}
+
+__host__ __device__ inline GemvPlan gemv_plan_for(int mt, int fmt, int k, int rt, int kc, int depth, int warps) {
+  GemvPlan p{};
+  p.warps = warps;
+  p.rt = rt;
+  p.kc = kc;
+  p.depth = depth;
+  p.sc_off = gemv_align16(rt * kc);
+  p.s2_off = p.sc_off + gemv_s1_window(rt, kc);
+  p.stage_bytes = gemv_align128(p.sc_off + gemv_sc_bytes(fmt, rt, kc));
+  // [act MT*K][warps x depth stages][barriers: warps x depth + 1][counter]
+  p.smem = gemv_align128(mt * k) + warps * depth * p.stage_bytes + 8 * (warps * depth + 1) + 16;
+  return p;
+}
+
+// Stage size: as many whole rows as fit `target` bytes (at most 32), else one
+// row in chunks of `target` (a multiple of 512) bytes.
+__host__ __device__ inline GemvPlan gemv_plan(int mt, int fmt, int k, int target, int depth, int warps) {
+  if (k <= target) {
+    int rt = target / k;
+    if (rt > kGemvMaxRowsPerTile) rt = kGemvMaxRowsPerTile;
+    return gemv_plan_for(mt, fmt, k, rt, k, depth, warps);
+  }
+  return gemv_plan_for(mt, fmt, k, 1, target & ~511, depth, warps);
 }
 
 __device__ __forceinline__ int dot16(const int4 w, const int4 x) {
@@ -87,317 +108,392 @@ __device__ __forceinline__ int dot16(const int4 w, const int4 x) {
   return p;
 }
 
-// Bytes of [src, src + bytes) that go by bulk copy: the whole 16-byte
-// multiple when src is 16-byte aligned, else none.
-__device__ __forceinline__ int bulk_part(const void* src, int bytes) {
-  return (reinterpret_cast<uintptr_t>(src) & 15u) == 0 ? (bytes & ~15) : 0;
+// Plan the copy of bytes [o0, o1) of a 16-byte-aligned array of `total`
+// bytes into dst as the 16-byte-aligned window [o0 & ~15, ...) around them,
+// one bulk copy; dst[(o0 & 15) + i] is then byte o0 + i. Only bytes past the
+// last whole 16 of the array (the final rows of a matrix) go by plain loads,
+// done here (by the lane with copy_tail) before the caller's arrive.
+struct GemvWindow {
+  const uint8_t* src;
+  uint8_t* dst;
+  uint32_t bytes;
+};
+__device__ __forceinline__ GemvWindow window_copy_plan(uint8_t* dst, const uint8_t* base, int64_t total, int64_t o0,
+                                                       int64_t o1, bool copy_tail) {
+  const int64_t w0 = o0 & ~int64_t(15);
+  const int64_t e16 = total & ~int64_t(15);
+  int64_t w1 = (o1 + 15) & ~int64_t(15);
+  if (w1 > e16) {
+    w1 = e16;
+    if (copy_tail)
+      for (int64_t b = (w0 > e16 ? w0 : e16); b < o1; ++b) dst[b - w0] = __ldg(base + b);
+  }
+  GemvWindow w{base + w0, dst, w1 > w0 ? static_cast<uint32_t>(w1 - w0) : 0u};
+  return w;
 }
 
-// Plain byte copy of the part bulk_part leaves (done before the arrive, so
-// the barrier's release orders it for the consumers).
-__device__ __forceinline__ void plain_tail(uint8_t* dst, const uint8_t* src, int from, int bytes) {
-  for (int b = from; b < bytes; ++b) dst[b] = __ldg(src + b);
+// One issued stage, as the issuing lane described it to its warp.
+struct GemvStage {
+  int64_t tile;  // -1: nothing issued
+  int chunk;
+};
+
+// Fused prologue: rotate and quantise the M token rows of x (bf16) into the
+// shared activation buffer, one fp32 scale per token, with the same
+// arithmetic as the standalone activation kernel (see act_quant.cuh): pass 1
+// finds each token's amax, pass 2 repeats the identical transform and
+// quantises. Every CTA does this for itself; CTA 0 writes the codes and scales
+// back when asked. Called by all threads.
+template <int MT>
+__device__ __forceinline__ void gemv_fused_act(const LinearArgs& a, int8_t* act, float* xscale, float* red) {
+  const int K = static_cast<int>(a.k);
+  const int M = static_cast<int>(a.m);
+  const int slots = K / kActSlot;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int iters = (slots + blockDim.x - 1) / blockDim.x;
+  float mx[MT];
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    mx[m] = 0.0f;
+    if (m >= M) continue;
+    const uint16_t* xr = a.x + static_cast<int64_t>(m) * K;
+    for (int j = 0; j < iters; ++j) {
+      const int s = threadIdx.x + j * blockDim.x;
+      float v[kActSlot];
+      if (s < slots) {
+        act_load_slot(xr + s * kActSlot, v, false);
+      } else {
+#pragma unroll
+        for (int i = 0; i < kActSlot; ++i) v[i] = 0.0f;
+      }
+      if (a.rotated) act_fwht_slot(v, lane);  // whole 8-lane groups are in or out
+      mx[m] = fmaxf(mx[m], act_slot_absmax(v));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx[m] = fmaxf(mx[m], __shfl_xor_sync(0xffffffffu, mx[m], o));
+    if (lane == 0) red[m * 32 + warp] = mx[m];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int m = 0; m < MT; ++m) {
+    if (m >= M) {
+      xscale[m] = 0.0f;
+      continue;
+    }
+    float amax = 0.0f;
+    for (int w = 0; w < nwarps; ++w) amax = fmaxf(amax, red[m * 32 + w]);
+    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    xscale[m] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+    const uint16_t* xr = a.x + static_cast<int64_t>(m) * K;
+    for (int j = 0; j < iters; ++j) {
+      const int s = threadIdx.x + j * blockDim.x;
+      float v[kActSlot];
+      if (s < slots) {
+        act_load_slot(xr + s * kActSlot, v, false);
+      } else {
+#pragma unroll
+        for (int i = 0; i < kActSlot; ++i) v[i] = 0.0f;
+      }
+      if (a.rotated) act_fwht_slot(v, lane);
+      if (s < slots) act_store_slot(act + m * K + s * kActSlot, v, inv);
+    }
+  }
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    if (a.xq_out) {
+      const int n16 = M * K / 16;
+      for (int i = threadIdx.x; i < n16; i += blockDim.x)
+        reinterpret_cast<int4*>(a.xq_out)[i] = reinterpret_cast<const int4*>(act)[i];
+    }
+    if (a.xs_out && threadIdx.x < M) a.xs_out[threadIdx.x] = xscale[threadIdx.x < MT ? threadIdx.x : 0];
+  }
 }
 
-template <int MT, int FMT, bool PARTIALS>
-__global__ void __launch_bounds__(kGemvThreads, 1)
-    gemv_kernel(const LinearArgs a, int stages, int64_t tiles_base, int64_t tiles_extra) {
-  using S = GemvShape<MT>;
+template <int MT, int RG, int FMT, bool PARTIALS, bool FUSED>
+__global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
+    gemv_kernel(const LinearArgs a, const GemvPlan p, int64_t tiles_base, int64_t tiles_extra) {
   constexpr int G = FMT == 0 ? kGroupTrunk : kGroupHead;
-  using Red = typename std::conditional<FMT == 0, long long, float>::type;
+  constexpr int LPB = G / 16;  // lanes per block within a 512-byte step
+  constexpr int kGemvUnroll = gemv_unroll(MT, RG);
 
   extern __shared__ __align__(128) uint8_t smem[];
   const int K = static_cast<int>(a.k);
   const int64_t N = a.n;
   const int M = static_cast<int>(a.m);
   const int ng = K / G;
-  const GemvSmem L = gemv_smem_layout(MT, FMT, K, stages, gemv_red_bytes<MT, FMT>());
-  const int slot_bytes = gemv_scale_slot_bytes(FMT, K);
-  int8_t* act = reinterpret_cast<int8_t*>(smem);
-  uint8_t* ring = smem + L.ring;
-  uint8_t* scl = smem + L.scales;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L.bars);
-  uint64_t* empty = full + stages;
-  uint64_t* sfull = empty + stages;
-  uint64_t* sempty = sfull + kGemvScaleSlots;
-  uint64_t* actbar = sempty + kGemvScaleSlots;
-  Red* red = reinterpret_cast<Red*>(smem + L.red);
-  // Set by any role whose bounded wait ran out; everyone then skips further
-  // waits but still reaches every barrier, so the CTA always finishes.
-  __shared__ volatile int s_abort;
-
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  int8_t* act = reinterpret_cast<int8_t*>(smem);
+  uint8_t* bufs = smem + gemv_align128(MT * K) + warp * p.depth * p.stage_bytes;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + gemv_align128(MT * K) + p.warps * p.depth * p.stage_bytes);
+  uint64_t* full = bars + warp * p.depth;
+  uint64_t* actbar = bars + p.warps * p.depth;
+  int* counter = reinterpret_cast<int*>(actbar + 1);
+
   const int64_t bid = blockIdx.x;
   const int64_t t0 = bid * tiles_base + (bid < tiles_extra ? bid : tiles_extra);
   const int64_t t1 = t0 + tiles_base + (bid < tiles_extra ? 1 : 0);
-  const int nchunks = (K + kGemvKC - 1) / kGemvKC;
+  const int nchunks = (K + p.kc - 1) / p.kc;
 
   if (threadIdx.x == 0) {
-    s_abort = 0;
-    for (int s = 0; s < stages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kGemvConsumerWarps);
-    }
-    for (int s = 0; s < kGemvScaleSlots; ++s) {
-      mbar_init(&sfull[s], 1);
-      mbar_init(&sempty[s], kGemvConsumerWarps);
-    }
+    for (int s = 0; s < p.warps * p.depth; ++s) mbar_init(&bars[s], 1);
     mbar_init(actbar, 1);
+    *counter = 0;
     fence_barrier_init();
   }
-  __syncthreads();
-
-  if (warp == kGemvConsumerWarps) {
-    // ---------------------------------------------------------- producer
-    if (lane == 0) {
-      const uint64_t pol = l2_policy_evict_first();
-      // the M token rows of activation codes, contiguous [M][K]
-      mbar_arrive_expect_tx(actbar, static_cast<uint32_t>(M * K));
-      bulk_g2s_default(act, a.xq, static_cast<uint32_t>(M * K), actbar);
-      uint32_t it = 0;
-      uint32_t lt = 0;
-      bool ok = true;
-      for (int64_t tile = t0; tile < t1 && ok; ++tile, ++lt) {
-        const int64_t row0 = tile * kGemvRows;
-        const int rows = static_cast<int>(min(static_cast<int64_t>(kGemvRows), N - row0));
-        if (!PARTIALS) {
-          const int ss = static_cast<int>(lt % kGemvScaleSlots);
-          const uint32_t suse = lt / kGemvScaleSlots;
-          if (s_abort || (suse > 0 && !mbar_wait(&sempty[ss], (suse - 1) & 1u, kDevErrGemvEmpty))) {
-            s_abort = 1;
-            ok = false;
-            break;
-          }
-          uint8_t* dst = scl + ss * slot_bytes;
-          const uint8_t* src0;
-          int bytes0;
-          if (FMT == 0) {
-            src0 = a.sub + row0 * ng;
-            bytes0 = rows * ng;
-          } else {
-            src0 = reinterpret_cast<const uint8_t*>(a.scale + row0 * ng);
-            bytes0 = rows * ng * 2;
-          }
-          const int nb0 = bulk_part(src0, bytes0);
-          plain_tail(dst, src0, nb0, bytes0);
-          int nb1 = 0;
-          const uint8_t* src1 = nullptr;
-          uint8_t* dst1 = dst + gemv_s2_offset(K);
-          if (FMT == 0) {
-            src1 = reinterpret_cast<const uint8_t*>(a.scale + row0);
-            nb1 = bulk_part(src1, rows * 2);
-            plain_tail(dst1, src1, nb1, rows * 2);
-          }
-          mbar_arrive_expect_tx(&sfull[ss], static_cast<uint32_t>(nb0 + nb1));
-          if (nb0) bulk_g2s(dst, src0, static_cast<uint32_t>(nb0), &sfull[ss], pol);
-          if (nb1) bulk_g2s(dst1, src1, static_cast<uint32_t>(nb1), &sfull[ss], pol);
-        }
-        for (int c = 0; c < nchunks; ++c) {
-          const int slot = static_cast<int>(it % stages);
-          const uint32_t use = it / stages;
-          if (s_abort || (use > 0 && !mbar_wait(&empty[slot], (use - 1) & 1u, kDevErrGemvEmpty))) {
-            s_abort = 1;
-            ok = false;
-            break;
-          }
-          const int len = min(kGemvKC, K - c * kGemvKC);
-          mbar_arrive_expect_tx(&full[slot], static_cast<uint32_t>(rows * len));
-          uint8_t* dst = ring + slot * kGemvStageBytes;
-          const int8_t* src = a.codes + row0 * K + c * kGemvKC;
-          for (int r = 0; r < rows; ++r)
-            bulk_g2s(dst + r * kGemvKC, src + static_cast<int64_t>(r) * K, static_cast<uint32_t>(len), &full[slot],
-                     pol);
-          ++it;
-        }
-      }
-      // never leave with a copy still landing in this CTA's shared memory
-      bool drained = mbar_wait(actbar, 0u, kDevErrGemvDrain);
-      const uint32_t first = it > static_cast<uint32_t>(stages) ? it - stages : 0u;
-      for (uint32_t j = first; j < it && drained; ++j)
-        drained = mbar_wait(&full[j % stages], (j / stages) & 1u, kDevErrGemvDrain);
-      if (!PARTIALS) {
-        const uint32_t sfirst = lt > static_cast<uint32_t>(kGemvScaleSlots) ? lt - kGemvScaleSlots : 0u;
-        for (uint32_t j = sfirst; j < lt && drained; ++j)
-          drained = mbar_wait(&sfull[j % kGemvScaleSlots], (j / kGemvScaleSlots) & 1u, kDevErrGemvDrain);
-      }
-    }
-    return;
-  }
-
-  // ------------------------------------------------------------ consumers
-  const int wr = warp % S::WR;
-  const int wk = warp / S::WR;
   // token rows past M are zero (their codes never reach an output anyway)
   {
     int4* pad = reinterpret_cast<int4*>(act + M * K);
     const int n16 = (MT - M) * K / 16;
-    for (int i = threadIdx.x; i < n16; i += kGemvConsumerWarps * 32) pad[i] = make_int4(0, 0, 0, 0);
+    for (int i = threadIdx.x; i < n16; i += blockDim.x) pad[i] = make_int4(0, 0, 0, 0);
   }
-  named_barrier(1, kGemvConsumerWarps * 32);
-  float xscale[MT];
+  __syncthreads();
+  if (!FUSED && threadIdx.x == 0) {
+    mbar_arrive_expect_tx(actbar, static_cast<uint32_t>(M * K));
+    bulk_g2s_default(act, a.xq, static_cast<uint32_t>(M * K), actbar);
+  }
+  const uint64_t pol = l2_policy_evict_first();
+
+  // ---- issuing (lane 0): claim work, fill stage buffer `b`
+  int64_t cur_tile = -1;  // tile whose chunks are being issued
+  int cur_chunk = 0;
+  GemvStage issued[kGemvMaxDepth];
+  uint32_t uses[kGemvMaxDepth];
 #pragma unroll
-  for (int m = 0; m < MT; ++m) xscale[m] = (!PARTIALS && m < M) ? a.xs[m] : 0.0f;
+  for (int b = 0; b < kGemvMaxDepth; ++b) {
+    issued[b].tile = -1;
+    issued[b].chunk = 0;
+    uses[b] = 0;
+  }
+  auto issue = [&](int b) {
+    // advance to the next (tile, chunk); lane 0 claims tiles, all lanes learn
+    int64_t tile = -1;
+    int chunk = 0;
+    if (cur_tile >= 0 && cur_chunk + 1 < nchunks) {
+      tile = cur_tile;
+      chunk = cur_chunk + 1;
+    } else {
+      int claimed = 0;
+      if (lane == 0) claimed = atomicAdd(counter, 1);
+      claimed = __shfl_sync(0xffffffffu, claimed, 0);
+      tile = t0 + claimed < t1 ? t0 + claimed : -1;
+    }
+    cur_tile = tile;
+    cur_chunk = chunk;
+    issued[b].tile = tile;
+    issued[b].chunk = chunk;
+    if (tile < 0) return;
+    // every lane computes the stage descriptor; lane 0 arms the barrier, then
+    // lanes 0, 1, 2 issue the codes, sub-scale and row-scale copies at once
+    const int64_t row0 = tile * p.rt;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(p.rt), N - row0));
+    const int len = min(p.kc, K - chunk * p.kc);
+    uint8_t* st = bufs + b * p.stage_bytes;
+    const int cbytes = rows * len;
+    GemvWindow w0{nullptr, nullptr, 0u}, w1{nullptr, nullptr, 0u};
+    if (!PARTIALS && lane < 3) {
+      const int gb = len / G;
+      const int64_t o0 = row0 * ng + chunk * (p.kc / G);  // first scale of the stage, in elements
+      if (FMT == 0) {
+        w0 = window_copy_plan(st + p.sc_off, a.sub, N * ng, o0, o0 + rows * gb, lane == 1);
+        // every chunk carries the row scales: the epilogue runs on the last
+        w1 = window_copy_plan(st + p.s2_off, reinterpret_cast<const uint8_t*>(a.scale), 2 * N, 2 * row0,
+                              2 * (row0 + rows), lane == 2);
+      } else {
+        w0 = window_copy_plan(st + p.sc_off, reinterpret_cast<const uint8_t*>(a.scale), 2 * N * ng, 2 * o0,
+                              2 * (o0 + rows * gb), lane == 1);
+      }
+    }
+    __syncwarp();  // plain tails (if any) are written before the arrive
+    if (lane == 0) mbar_arrive_expect_tx(&full[b], static_cast<uint32_t>(cbytes) + w0.bytes + w1.bytes);
+    __syncwarp();
+    if (lane == 0) {
+      const int8_t* src = a.codes + row0 * K + chunk * p.kc;  // rows x len, contiguous
+      for (int off = 0; off < cbytes; off += kGemvMaxCopy)
+        bulk_g2s(st + off, src + off, static_cast<uint32_t>(min(kGemvMaxCopy, cbytes - off)), &full[b], pol);
+    } else if (lane == 1 && w0.bytes) {
+      bulk_g2s(w0.dst, w0.src, w0.bytes, &full[b], pol);
+    } else if (lane == 2 && w1.bytes) {
+      bulk_g2s(w1.dst, w1.src, w1.bytes, &full[b], pol);
+    }
+  };
+
+  for (int b = 0; b < p.depth; ++b) issue(b);
+
+  // activation codes: computed here (fused) while the first stages stream,
+  // or already on their way by bulk copy
+  float xscale[MT];
+  bool failed = false;  // warp-uniform: a wait ran out; stop computing
+  if (FUSED) {
+    __shared__ float red[MT * 32];
+    gemv_fused_act<MT>(a, act, xscale, red);
+  } else {
+#pragma unroll
+    for (int m = 0; m < MT; ++m) xscale[m] = (!PARTIALS && m < M) ? a.xs[m] : 0.0f;
+    const bool ok = mbar_wait(actbar, 0u, kDevErrGemvFull);
+    failed = !__all_sync(0xffffffffu, ok);
+  }
   const float rot = a.rotated ? 0.0078125f : 1.0f;
 
-  bool failed = false;  // warp-uniform
-  {
-    bool bad = s_abort != 0;
-    if (!bad) bad = !mbar_wait(actbar, 0u, kDevErrGemvFull);
-    failed = __any_sync(0xffffffffu, bad);
-    if (failed && lane == 0) s_abort = 1;
-  }
-
-  uint32_t it = 0;
-  uint32_t lt = 0;
-  int par = 0;
-  for (int64_t tile = t0; tile < t1; ++tile, ++lt, par ^= 1) {
-    const int64_t wrow0 = tile * kGemvRows + wr * S::RG;  // this warp's first row
-    const int ss = static_cast<int>(lt % kGemvScaleSlots);
-    const uint8_t* ts = scl + ss * slot_bytes;
-    if (!PARTIALS && !failed) {
-      bool bad = s_abort != 0;
-      if (!bad) bad = !mbar_wait(&sfull[ss], (lt / kGemvScaleSlots) & 1u, kDevErrGemvFull);
-      failed = __any_sync(0xffffffffu, bad);
-      if (failed && lane == 0) s_abort = 1;
+  // Sums of the row group in flight: int64 (trunk) or fp32 (lm_head). They
+  // carry across chunks only for one-row tiles; whole-row tiles have one chunk.
+  long long racc[RG][MT];
+  float facc[RG][MT];
+  int b = 0;
+  while (issued[b].tile >= 0) {
+    const int64_t tile = issued[b].tile;
+    const int chunk = issued[b].chunk;
+    if (!failed) {
+      const bool ok = mbar_wait(&full[b], uses[b] & 1u, kDevErrGemvFull);
+      failed = !__all_sync(0xffffffffu, ok);
     }
-    long long acc64[S::RG][MT];
-    float accf[S::RG][MT];
+    const uint8_t* st = bufs + b * p.stage_bytes;
+    const int64_t row0 = tile * p.rt;
+    const int rows = static_cast<int>(min(static_cast<int64_t>(p.rt), N - row0));
+    const int len = min(p.kc, K - chunk * p.kc);
+    const int gb = len / G;
+    // scales start inside their 16-byte window (see window_copy_plan)
+    const int64_t so = row0 * ng + chunk * (p.kc / G);
+    const uint8_t* sc = st + p.sc_off + (FMT == 0 ? (so & 15) : ((2 * so) & 15));
+    const uint16_t* s2p = reinterpret_cast<const uint16_t*>(st + p.s2_off + ((2 * row0) & 15));
+    const int nsteps = (len + 511) / 512;
+    for (int r0 = 0; r0 < rows; r0 += RG) {
+      if (chunk == 0) {
 #pragma unroll
-    for (int i = 0; i < S::RG; ++i)
-#pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        acc64[i][m] = 0;
-        accf[i][m] = 0.0f;
-      }
-    for (int c = 0; c < nchunks; ++c, ++it) {
-      const int slot = static_cast<int>(it % stages);
-      const int len = min(kGemvKC, K - c * kGemvKC);
-      if (!failed) {
-        bool bad = s_abort != 0;
-        if (!bad) bad = !mbar_wait(&full[slot], (it / stages) & 1u, kDevErrGemvFull);
-        failed = __any_sync(0xffffffffu, bad);
-        if (failed && lane == 0) s_abort = 1;
-      }
-      const uint8_t* stage = ring + slot * kGemvStageBytes;
-      int acc32[S::RG][MT];
-#pragma unroll
-      for (int i = 0; i < S::RG; ++i)
-#pragma unroll
-        for (int m = 0; m < MT; ++m) acc32[i][m] = 0;
-#pragma unroll
-      for (int u = 0; u < S::SPW; ++u) {
-        const int o = (wk + S::WK * u) * 512 + lane * 16;
-        const bool valid = !failed && o < len;  // uniform per 256-byte half-warp
-        const int kk = c * kGemvKC + o;
-        const int g = kk / G;
-        int4 xv[MT];
-#pragma unroll
-        for (int m = 0; m < MT; ++m)
-          xv[m] = valid ? *reinterpret_cast<const int4*>(act + m * K + kk) : make_int4(0, 0, 0, 0);
-#pragma unroll
-        for (int i = 0; i < S::RG; ++i) {
-          if (wrow0 + i >= N) continue;  // warp-uniform
-          const int rl = wr * S::RG + i;  // row within the tile
-          const int4 wv = valid ? *reinterpret_cast<const int4*>(stage + rl * kGemvKC + o) : make_int4(0, 0, 0, 0);
-          int s1 = 0;
-          float sf = 0.0f;
-          if (!PARTIALS && valid) {
-            if (FMT == 0)
-              s1 = ts[rl * ng + g];
-            else
-              sf = bf16_bits_to_float(reinterpret_cast<const uint16_t*>(ts)[rl * ng + g]);
-          }
+        for (int i = 0; i < RG; ++i)
 #pragma unroll
           for (int m = 0; m < MT; ++m) {
-            int p = dot16(wv, xv[m]);
-            if (PARTIALS) {
-              // 16 lanes (trunk) or 8 lanes (lm_head) make one block
+            racc[i][m] = 0;
+            facc[i][m] = 0.0f;
+          }
+      }
+      int acc32[RG][MT];
 #pragma unroll
-              for (int off = 1; off < G / 16; off <<= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
-              if (valid && m < M && (lane & (G / 16 - 1)) == 0)
-                a.partials[(static_cast<int64_t>(m) * N + wrow0 + i) * ng + g] = p;
-            } else if (FMT == 0) {
-              acc32[i][m] += s1 * p;  // <= 255 * 16 * 127^2 per step, <= 4 steps
-            } else {
-              accf[i][m] = fmaf(static_cast<float>(p), sf, accf[i][m]);
+      for (int i = 0; i < RG; ++i)
+#pragma unroll
+        for (int m = 0; m < MT; ++m) acc32[i][m] = 0;
+      int since = 0;
+      for (int t0s = 0; t0s < nsteps; t0s += kGemvUnroll) {
+        // loads for kGemvUnroll steps first, then the dot products
+        int4 xv[kGemvUnroll][MT];
+        int4 wv[kGemvUnroll][RG];
+        int s1v[kGemvUnroll][RG];
+        float sfv[kGemvUnroll][RG];
+#pragma unroll
+        for (int u = 0; u < kGemvUnroll; ++u) {
+          const int o = (t0s + u) * 512 + lane * 16;
+          const bool valid = !failed && o < len;  // uniform per 256-byte half-warp
+          const int kk = chunk * p.kc + o;
+#pragma unroll
+          for (int m = 0; m < MT; ++m)
+            xv[u][m] = valid ? *reinterpret_cast<const int4*>(act + m * K + kk) : make_int4(0, 0, 0, 0);
+#pragma unroll
+          for (int i = 0; i < RG; ++i) {
+            const int rl = r0 + i;
+            const bool vr = valid && rl < rows;
+            wv[u][i] = vr ? *reinterpret_cast<const int4*>(st + rl * len + o) : make_int4(0, 0, 0, 0);
+            s1v[u][i] = 0;
+            sfv[u][i] = 0.0f;
+            if (!PARTIALS && vr) {
+              if (FMT == 0)
+                s1v[u][i] = sc[rl * gb + o / G];
+              else
+                sfv[u][i] = bf16_bits_to_float(reinterpret_cast<const uint16_t*>(sc)[rl * gb + o / G]);
             }
           }
         }
+#pragma unroll
+        for (int u = 0; u < kGemvUnroll; ++u) {
+#pragma unroll
+          for (int i = 0; i < RG; ++i) {
+#pragma unroll
+            for (int m = 0; m < MT; ++m) {
+              int q = dot16(wv[u][i], xv[u][m]);
+              if (PARTIALS) {
+                // LPB lanes make one block: 16 (trunk) or 8 (lm_head)
+#pragma unroll
+                for (int off = 1; off < LPB; off <<= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
+                const int o = (t0s + u) * 512 + lane * 16;
+                if (!failed && o < len && r0 + i < rows && m < M && (lane & (LPB - 1)) == 0)
+                  a.partials[(static_cast<int64_t>(m) * N + row0 + r0 + i) * ng + (chunk * p.kc + o) / G] = q;
+              } else if (FMT == 0) {
+                acc32[i][m] += s1v[u][i] * q;  // |s1 * q| <= 255 * 16 * 127^2 < 2^26
+              } else {
+                facc[i][m] = fmaf(static_cast<float>(q), sfv[u][i], facc[i][m]);
+              }
+            }
+          }
+        }
+        if (FMT == 0 && !PARTIALS) {
+          since += kGemvUnroll;
+          if (since >= 16) {  // 16 steps < 2^30: fold before int32 can overflow
+            since = 0;
+#pragma unroll
+            for (int i = 0; i < RG; ++i)
+#pragma unroll
+              for (int m = 0; m < MT; ++m) {
+                racc[i][m] += acc32[i][m];
+                acc32[i][m] = 0;
+              }
+          }
+        }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[slot]);
       if (FMT == 0 && !PARTIALS) {
 #pragma unroll
-        for (int i = 0; i < S::RG; ++i)
+        for (int i = 0; i < RG; ++i)
 #pragma unroll
-          for (int m = 0; m < MT; ++m) acc64[i][m] += acc32[i][m];
+          for (int m = 0; m < MT; ++m) racc[i][m] += acc32[i][m];
       }
-    }
-    if (PARTIALS) continue;
-
-    // ------------------------------------------------------------ epilogue
-    Red tot[S::RG][MT];
+      // ---- epilogue once the tile's last chunk is in
+      if (!PARTIALS && chunk == nchunks - 1) {
+        uint16_t s2b[RG];
 #pragma unroll
-    for (int i = 0; i < S::RG; ++i)
+        for (int i = 0; i < RG; ++i)
+          s2b[i] = (FMT == 0 && r0 + i < rows) ? s2p[r0 + i] : 0;
 #pragma unroll
-      for (int m = 0; m < MT; ++m) {
-        Red v;
-        if (FMT == 0)
-          v = acc64[i][m];
-        else
-          v = accf[i][m];
+        for (int i = 0; i < RG; ++i) {
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-        tot[i][m] = v;
-      }
-    const uint16_t* s2 = reinterpret_cast<const uint16_t*>(ts + gemv_s2_offset(K));
-    if (S::WK > 1) {
-      Red* rb = red + par * (S::WK * S::WR * S::RG * MT);
-      if (lane == 0) {
+          for (int m = 0; m < MT; ++m) {
+            float yv;
+            if (FMT == 0) {
+              long long v = racc[i][m];
 #pragma unroll
-        for (int i = 0; i < S::RG; ++i)
+              for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+              yv = __ll2float_rn(v) * xscale[m] * bf16_bits_to_float(s2b[i]) * rot;
+            } else {
+              float v = facc[i][m];
 #pragma unroll
-          for (int m = 0; m < MT; ++m) rb[((wk * S::WR + wr) * S::RG + i) * MT + m] = tot[i][m];
-      }
-      named_barrier(1, kGemvConsumerWarps * 32);
-      if (wk == 0 && lane < S::RG * MT) {
-        const int i = lane / MT;
-        const int m = lane % MT;
-        Red v = 0;
-#pragma unroll
-        for (int w = 0; w < S::WK; ++w) v += rb[((w * S::WR + wr) * S::RG + i) * MT + m];
-        const int64_t row = wrow0 + i;
-        if (!failed && m < M && row < N) {
-          float yv;
-          if (FMT == 0)
-            yv = __ll2float_rn(static_cast<long long>(v)) * xscale[m] * bf16_bits_to_float(s2[wr * S::RG + i]) * rot;
-          else
-            yv = static_cast<float>(v) * xscale[m] * rot;
-          a.y[static_cast<int64_t>(m) * N + row] = float_to_bf16_bits_rn(yv);
-        }
-      }
-    } else if (lane == 0 && !failed) {
-#pragma unroll
-      for (int i = 0; i < S::RG; ++i) {
-        const int64_t row = wrow0 + i;
-        if (row >= N) continue;
-#pragma unroll
-        for (int m = 0; m < MT; ++m) {
-          if (m >= M) continue;
-          float yv;
-          if (FMT == 0)
-            yv = __ll2float_rn(static_cast<long long>(tot[i][m])) * xscale[m] *
-                 bf16_bits_to_float(s2[wr * S::RG + i]) * rot;
-          else
-            yv = static_cast<float>(tot[i][m]) * xscale[m] * rot;
-          a.y[static_cast<int64_t>(m) * N + row] = float_to_bf16_bits_rn(yv);
+              for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+              yv = v * xscale[m] * rot;
+            }
+            if (lane == i * MT + m && !failed && r0 + i < rows && m < M)
+              a.y[static_cast<int64_t>(m) * N + row0 + r0 + i] = float_to_bf16_bits_rn(yv);
+          }
         }
       }
     }
+    // the buffer is consumed: refill it (the chunk's data is no longer read)
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sempty[ss]);  // this warp is done with the tile's scales
+    uses[b] += 1;
+    if (!failed) {
+      issue(b);
+    } else {
+      issued[b].tile = -1;
+    }
+    b = b + 1 == p.depth ? 0 : b + 1;
+    if (failed) {
+      // drain: never leave with a copy still landing in this warp's buffers
+      for (int j = 0; j < p.depth; ++j)
+        if (issued[j].tile >= 0) {
+          mbar_wait(&full[j], uses[j] & 1u, kDevErrGemvDrain);
+          issued[j].tile = -1;
+        }
+      break;
+    }
   }
+  if (!FUSED && threadIdx.x == 0) mbar_wait(actbar, 0u, kDevErrGemvDrain);  // the shared copy has landed
 }
 
 }  // namespace iq8r

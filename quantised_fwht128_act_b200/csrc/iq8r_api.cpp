@@ -36,6 +36,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 constexpr int64_t kMaxK = int64_t(1) << 30;
 constexpr int64_t kMaxGridRows = (int64_t(1) << 31) - 1;
+// iq8r_linear_bf16 fuses the activation quantiser into the GEMV up to this
+// many activation elements (M * K); beyond it two launches are cheaper.
+constexpr int64_t kFuseMaxElems = 16384;
 
 iq8r_status check_weight(const iq8r_weight* w, const char* fn) {
   if (!w) return fail(IQ8R_ERR_INVALID_ARG, "%s: weight is NULL", fn);
@@ -50,8 +53,8 @@ iq8r_status check_weight(const iq8r_weight* w, const char* fn) {
   if (!w->codes || !w->scale) return fail(IQ8R_ERR_INVALID_ARG, "%s: weight codes or scale is NULL", fn);
   if (w->fmt == IQ8R_FMT_G256_U8_BF16 && !w->sub_scale)
     return fail(IQ8R_ERR_INVALID_ARG, "%s: the trunk format needs sub_scale", fn);
-  if (!aligned16(w->codes) || !aligned16(w->scale))
-    return fail(IQ8R_ERR_INVALID_ARG, "%s: weight codes and scale must be 16-byte aligned", fn);
+  if (!aligned16(w->codes) || !aligned16(w->scale) || (w->sub_scale && !aligned16(w->sub_scale)))
+    return fail(IQ8R_ERR_INVALID_ARG, "%s: weight codes, sub_scale and scale must be 16-byte aligned", fn);
   return IQ8R_OK;
 }
 
@@ -166,6 +169,42 @@ iq8r_status iq8r_linear_ex(const int8_t* xq, const float* x_scale, int64_t m, co
   iq8r::LinearArgs a = make_args(xq, x_scale, m, w);
   a.y = y_bf16;
   return run_linear(a, path, fn, stream);
+}
+
+iq8r_status iq8r_linear_bf16(const uint16_t* x_bf16, int64_t m, const iq8r_weight* w, uint16_t* y_bf16,
+                             int8_t* xq_out, float* x_scale_out, cudaStream_t stream) {
+  const char* fn = "iq8r_linear_bf16";
+  iq8r_status st = check_weight(w, fn);
+  if (st != IQ8R_OK) return st;
+  if (m < 0 || m > kMaxGridRows) return fail(IQ8R_ERR_INVALID_ARG, "%s: m = %lld out of range", fn, (long long)m);
+  if (w->k % iq8r::kRot) return fail(IQ8R_ERR_INVALID_ARG, "%s: k must be a multiple of 128", fn);
+  if (m == 0) return ok();
+  if (!x_bf16 || !y_bf16) return fail(IQ8R_ERR_INVALID_ARG, "%s: NULL buffer", fn);
+  if (!aligned16(x_bf16) || !aligned16(y_bf16) || (xq_out && !aligned16(xq_out)))
+    return fail(IQ8R_ERR_INVALID_ARG, "%s: x, y and xq_out must be 16-byte aligned", fn);
+  std::string why;
+  // One launch when the activation is small enough that every CTA redoing
+  // its rotation is cheap, or when there is nowhere to stage the codes.
+  const bool small = m * w->k <= kFuseMaxElems;
+  const bool staged = xq_out && x_scale_out;
+  if (m <= 8 && (small || !staged) && iq8r::gemv_supported(w->k, &why)) {
+    // one launch: every CTA rotates and quantises x itself, then streams W
+    iq8r::LinearArgs a = make_args(nullptr, nullptr, m, w);
+    a.y = y_bf16;
+    a.x = x_bf16;
+    a.xq_out = xq_out;
+    a.xs_out = x_scale_out;
+    const cudaError_t e = iq8r::launch_gemv(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return ok();
+  }
+  if (!staged)
+    return fail(IQ8R_ERR_INVALID_ARG, "%s: m > 8 needs xq_out and x_scale_out (the codes are staged there)", fn);
+  cudaError_t e = iq8r::launch_act_quant(x_bf16, m, w->k, w->rotated, xq_out, x_scale_out, stream);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  iq8r::LinearArgs a = make_args(xq_out, x_scale_out, m, w);
+  a.y = y_bf16;
+  return run_linear(a, IQ8R_PATH_AUTO, fn, stream);
 }
 
 iq8r_status iq8r_linear(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w, uint16_t* y_bf16,

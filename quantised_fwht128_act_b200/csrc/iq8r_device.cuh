@@ -16,9 +16,11 @@ namespace iq8r {
 // it through iq8r_get_device_error.
 __device__ uint32_t g_device_error;
 
-// Upper bound on any single wait inside a kernel. Waits normally last
-// nanoseconds to microseconds; a second means the partner role is gone.
-constexpr uint64_t kWaitLimitNs = 1000ull * 1000ull * 1000ull;
+// Upper bound on any single wait inside a kernel, in SM clock cycles
+// (about a second at B200 clocks). Waits normally last nanoseconds to
+// microseconds; running out means the partner role is gone. The SM's own
+// cycle counter is used because it is cheap to read inside a polling loop.
+constexpr uint64_t kWaitLimitCycles = 2000ull * 1000ull * 1000ull;
 
 __device__ __forceinline__ void set_device_error(uint32_t code) {
   atomicCAS(&g_device_error, 0u, code);
@@ -26,12 +28,6 @@ __device__ __forceinline__ void set_device_error(uint32_t code) {
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ uint64_t global_timer_ns() {
-  uint64_t t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -53,29 +49,33 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
                : "memory");
 }
 
+// One poll of the barrier. A thread whose phase is not complete yet may be
+// suspended (not spinning, so it leaves issue slots to working warps) for up
+// to kSuspendHintNs before the poll reports "not yet".
+constexpr uint32_t kSuspendHintNs = 20000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_addr(bar)), "r"(parity)
+      : "r"(smem_addr(bar)), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
 
 // Wait for the phase with the given parity to complete, for at most
-// limit_ns. On timeout: record `code` and return false.
+// limit_cycles SM cycles. On timeout: record `code` and return false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t code,
-                                          uint64_t limit_ns = kWaitLimitNs) {
+                                          uint64_t limit_cycles = kWaitLimitCycles) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = global_timer_ns();
+  const long long t0 = clock64();
   while (true) {
 #pragma unroll 1
-    for (int i = 0; i < 32; ++i)
+    for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > limit_ns) {
+    if (static_cast<uint64_t>(clock64() - t0) > limit_cycles) {
       set_device_error(code);
       return false;
     }

@@ -41,6 +41,10 @@ struct LinearArgs {
   const uint16_t* scale; // [n] (G256) or [n][k/128] (G128)
   uint16_t* y;           // [m][n] bf16, or nullptr in partials mode
   int32_t* partials;     // [m][n][k/G] in partials mode, else nullptr
+  // fused mode (x given): the kernel rotates and quantises x itself
+  const uint16_t* x;     // [m][k] bf16, or nullptr
+  int8_t* xq_out;        // [m][k] codes written back when not null
+  float* xs_out;         // [m] scales written back when not null
 };
 
 // Launchers (iq8r_kernels.cu). They validate nothing: the ABI layer has.

@@ -14,6 +14,7 @@ namespace iq8r {
 namespace {
 
 constexpr int kMaxDevices = 64;
+constexpr int kGemvY = 0, kGemvPartials = 1, kGemvFused = 2;  // what a GEMV launch produces
 
 struct DeviceInfo {
   int num_sms = 0;
@@ -58,34 +59,62 @@ cudaError_t ensure_smem(Kernel kernel, int bytes, std::atomic<int>* configured) 
 }
 
 // Static shared memory and alignment slack kept out of the dynamic budget.
-constexpr int kSmemReserve = 1024;
+constexpr int kSmemReserve = 2048;
 
-template <int MT, int FMT, bool PARTIALS>
-cudaError_t launch_gemv_t(const LinearArgs& a, const DeviceInfo& d, cudaStream_t stream) {
-  const int k = static_cast<int>(a.k);
-  const int red = gemv_red_bytes<MT, FMT>();
+// Stage size and depth for a token tile of `mt`: the shared memory left after
+// the activation codes is split over the warps; each gets two or more stages
+// of up to 16 KB of codes (whole rows when they fit). rt == 0: no fit.
+GemvPlan gemv_choose(int mt, int fmt, int k, const DeviceInfo& d) {
+  GemvPlan none{};
+  const int warps = gemv_warps(mt);
   const int budget = d.smem_optin - kSmemReserve;
-  int stages = kGemvMaxStages;
-  while (stages >= 2 && gemv_smem_layout(MT, FMT, k, stages, red).total > budget) --stages;
-  if (stages < 2) return cudaErrorInvalidConfiguration;
-  const int smem = gemv_smem_layout(MT, FMT, k, stages, red).total;
-  auto kernel = gemv_kernel<MT, FMT, PARTIALS>;
+  const int avail = budget - gemv_align128(mt * k) - 8 * (warps * kGemvMaxDepth + 1) - 16;
+  if (avail <= 0) return none;
+  const int per_warp = avail / warps;
+  for (int target = std::min(16 * 1024, (per_warp / 2) & ~511); target >= 512; target -= 512) {
+    GemvPlan p = gemv_plan(mt, fmt, k, target, 2, warps);
+    const int depth = std::min(kGemvMaxDepth, per_warp / p.stage_bytes);
+    if (depth < 2) continue;
+    p = gemv_plan(mt, fmt, k, target, depth, warps);
+    if (p.smem <= budget) return p;
+  }
+  return none;
+}
+
+template <int MT, int RG, int FMT, int MODE>
+cudaError_t launch_gemv_t(const LinearArgs& a, const GemvPlan& p, const DeviceInfo& d, cudaStream_t stream) {
+  auto kernel = gemv_kernel<MT, RG, FMT, MODE == kGemvPartials, MODE == kGemvFused>;
   static std::atomic<int> configured[kMaxDevices];
-  cudaError_t e = ensure_smem(kernel, smem, configured);
+  cudaError_t e = ensure_smem(kernel, p.smem, configured);
   if (e != cudaSuccess) return e;
-  const int64_t tiles = (a.n + kGemvRows - 1) / kGemvRows;
+  const int64_t tiles = (a.n + p.rt - 1) / p.rt;
   const int64_t grid = std::min<int64_t>(d.num_sms, tiles);
-  kernel<<<static_cast<unsigned>(grid), kGemvThreads, smem, stream>>>(a, stages, tiles / grid, tiles % grid);
+  kernel<<<static_cast<unsigned>(grid), p.warps * 32, p.smem, stream>>>(a, p, tiles / grid, tiles % grid);
   return cudaGetLastError();
 }
 
-template <int FMT, bool PARTIALS>
+template <int FMT, int MODE>
 cudaError_t launch_gemv_mt(const LinearArgs& a, int mt, const DeviceInfo& d, cudaStream_t stream) {
+  const GemvPlan p = gemv_choose(mt, FMT, static_cast<int>(a.k), d);
+  if (p.rt == 0) return cudaErrorInvalidConfiguration;
+  // rows computed together: up to 1, 2 or 4 by token count, never past a tile
+  const int pref = mt <= 2 ? 2 : 4;
+  const int rg = std::min(pref, p.rt) >= 4 ? 4 : (std::min(pref, p.rt) >= 2 ? 2 : 1);
   switch (mt) {
-    case 1: return launch_gemv_t<1, FMT, PARTIALS>(a, d, stream);
-    case 2: return launch_gemv_t<2, FMT, PARTIALS>(a, d, stream);
-    case 4: return launch_gemv_t<4, FMT, PARTIALS>(a, d, stream);
-    default: return launch_gemv_t<8, FMT, PARTIALS>(a, d, stream);
+    case 1:
+      return rg == 1 ? launch_gemv_t<1, 1, FMT, MODE>(a, p, d, stream)
+                     : launch_gemv_t<1, 2, FMT, MODE>(a, p, d, stream);
+    case 2:
+      return rg == 1 ? launch_gemv_t<2, 1, FMT, MODE>(a, p, d, stream)
+                     : launch_gemv_t<2, 2, FMT, MODE>(a, p, d, stream);
+    case 4:
+      return rg == 1   ? launch_gemv_t<4, 1, FMT, MODE>(a, p, d, stream)
+             : rg == 2 ? launch_gemv_t<4, 2, FMT, MODE>(a, p, d, stream)
+                       : launch_gemv_t<4, 4, FMT, MODE>(a, p, d, stream);
+    default:
+      return rg == 1   ? launch_gemv_t<8, 1, FMT, MODE>(a, p, d, stream)
+             : rg == 2 ? launch_gemv_t<8, 2, FMT, MODE>(a, p, d, stream)
+                       : launch_gemv_t<8, 4, FMT, MODE>(a, p, d, stream);
   }
 }
 
@@ -99,10 +128,8 @@ int next_pow2(int v) {
 // two-stage ring.
 int gemv_max_mt(int64_t k, const DeviceInfo& d) {
   if (k > (int64_t(1) << 24)) return 0;
-  for (int mt = 8; mt >= 1; mt >>= 1) {
-    const int need = gemv_smem_layout(mt, 1, static_cast<int>(k), 2, 2 * 8 * 8 * 8).total;
-    if (need <= d.smem_optin - kSmemReserve) return mt;
-  }
+  for (int mt = 8; mt >= 1; mt >>= 1)
+    if (gemv_choose(mt, 0, static_cast<int>(k), d).rt && gemv_choose(mt, 1, static_cast<int>(k), d).rt) return mt;
   return 0;
 }
 
@@ -148,13 +175,21 @@ cudaError_t launch_gemv(const LinearArgs& a, cudaStream_t stream) {
     s.xq = a.xq + m0 * a.k;
     if (a.xs) s.xs = a.xs + m0;
     if (a.y) s.y = a.y + m0 * a.n;
+    if (a.x) s.x = a.x + m0 * a.k;
+    if (a.xq_out) s.xq_out = a.xq_out + m0 * a.k;
+    if (a.xs_out) s.xs_out = a.xs_out + m0;
     if (a.partials) s.partials = a.partials + m0 * a.n * ng;
     const int mt = next_pow2(mg);
     const bool part = a.partials != nullptr;
+    const int mode = part ? kGemvPartials : (a.x ? kGemvFused : kGemvY);
     if (a.fmt == 0)
-      e = part ? launch_gemv_mt<0, true>(s, mt, d, stream) : launch_gemv_mt<0, false>(s, mt, d, stream);
+      e = mode == kGemvPartials ? launch_gemv_mt<0, kGemvPartials>(s, mt, d, stream)
+          : mode == kGemvFused  ? launch_gemv_mt<0, kGemvFused>(s, mt, d, stream)
+                                : launch_gemv_mt<0, kGemvY>(s, mt, d, stream);
     else
-      e = part ? launch_gemv_mt<1, true>(s, mt, d, stream) : launch_gemv_mt<1, false>(s, mt, d, stream);
+      e = mode == kGemvPartials ? launch_gemv_mt<1, kGemvPartials>(s, mt, d, stream)
+          : mode == kGemvFused  ? launch_gemv_mt<1, kGemvFused>(s, mt, d, stream)
+                                : launch_gemv_mt<1, kGemvY>(s, mt, d, stream);
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
@@ -184,19 +219,20 @@ namespace {
 
 // One thread waits on a barrier that nothing will ever arrive on; the
 // bounded wait must give up after limit_ns and record the self-test code.
-__global__ void wait_selftest_kernel(uint64_t limit_ns) {
+__global__ void wait_selftest_kernel(uint64_t limit_cycles) {
   __shared__ uint64_t bar;
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     fence_barrier_init();
-    mbar_wait(&bar, 0u, kDevErrSelftest, limit_ns);
+    mbar_wait(&bar, 0u, kDevErrSelftest, limit_cycles);
   }
 }
 
 }  // namespace
 
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream) {
-  wait_selftest_kernel<<<1, 32, 0, stream>>>(limit_ns);
+  // cycles at no more than 2 GHz: the wait lasts at most about limit_ns
+  wait_selftest_kernel<<<1, 32, 0, stream>>>(2 * limit_ns);
   return cudaGetLastError();
 }
 

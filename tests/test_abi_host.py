@@ -148,6 +148,7 @@ def test_gpu_calls_reject_bad_arguments_before_any_launch(L):
         weight(codes=0),
         weight(sub_scale=0),
         weight(codes=(1 << 20) + 4),
+        weight(sub_scale=(1 << 21) + 8),
     ]
     for w in bad:
         assert lin(w) == iq8r.IQ8R_ERR_INVALID_ARG, iq8r.iq8r_last_error()

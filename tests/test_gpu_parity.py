@@ -263,3 +263,52 @@ def test_bounded_wait_reports_timeout_and_context_survives():
     x, _, fmt, packed, W = case("pr1")
     y64 = oracle_linear(x, fmt, packed)
     check_output(gpu_linear(x, W), y64)
+
+
+# ------------------------------------------------------- fused bf16 entry
+
+@pytest.mark.parametrize("name,m,n,k", [("pr1", None, None, None), ("decode", None, None, None),
+                                        ("verify8", None, None, None), ("decode", 3, 1000, 768),
+                                        ("decode", 5, 37, 2304), ("decode", 7, 40, 17408)])
+def test_linear_bf16_fused_matches_two_call_path(name, m, n, k):
+    """One-launch act + GEMV: codes and scales bit-exact against the oracle,
+    y bit-identical to the two-call path and within tolerance of the oracle."""
+    x, _, fmt, packed, W = case(name, m=m, n=n, k=k, seed=None if m is None else 31 + m + n)
+    xd = dev_bf16(x)
+    xq_out = torch.empty(x.shape, dtype=torch.int8, device="cuda")
+    xs_out = torch.empty((x.shape[0],), dtype=torch.float32, device="cuda")
+    y = iq8r.iq8r_linear_bf16(xd, W, xq_out=xq_out, x_scale_out=xs_out)
+    torch.cuda.synchronize()
+    q, a = oracle.act_quant(x)
+    assert np.array_equal(xq_out.cpu().numpy(), q)
+    assert np.array_equal(xs_out.cpu().numpy().view(np.uint32), a.view(np.uint32))
+    y2 = gpu_linear(x, W)
+    assert np.array_equal(host_bits(y), y2)
+    y64 = oracle_linear(x, fmt, packed)
+    check_output(host_bits(y), y64, oracle.linear_bf16(y64))
+
+
+def test_linear_bf16_lm_head_and_no_outputs():
+    x, _, fmt, packed, W = case("lm_head8", m=8, n=2000, k=5120, seed=45)
+    y = iq8r.iq8r_linear_bf16(dev_bf16(x), W)
+    torch.cuda.synchronize()
+    y64 = oracle_linear(x, fmt, packed)
+    check_output(host_bits(y), y64, oracle.linear_bf16(y64))
+
+
+def test_linear_bf16_large_m_stages_codes():
+    x, _, fmt, packed, W = case("verify16")
+    xq_out = torch.empty(x.shape, dtype=torch.int8, device="cuda")
+    xs_out = torch.empty((x.shape[0],), dtype=torch.float32, device="cuda")
+    y = iq8r.iq8r_linear_bf16(dev_bf16(x), W, xq_out=xq_out, x_scale_out=xs_out)
+    torch.cuda.synchronize()
+    q, a = oracle.act_quant(x)
+    assert np.array_equal(xq_out.cpu().numpy(), q)
+    y64 = oracle_linear(x, fmt, packed)
+    check_output(host_bits(y), y64, oracle.linear_bf16(y64))
+    # without staging buffers M > 8 is refused, not silently allocated
+    w = W._struct()
+    import ctypes
+    st = iq8r.lib().iq8r_linear_bf16(dev_bf16(x).data_ptr(), x.shape[0], ctypes.byref(w), y.data_ptr(), None, None,
+                                      torch.cuda.current_stream().cuda_stream)
+    assert st == iq8r.IQ8R_ERR_INVALID_ARG
