@@ -1,0 +1,361 @@
+// IQ8R linear on the 5th-generation tensor cores (tcgen05, kind::i8) for
+// prefill-sized M: the one place the layer is a dense contraction.
+//
+// y[m][n] = a[m] * s2[n] / 128 * sum_g s1[n][g] * P[m][n][g] (trunk) or
+// a[m] / 128 * sum_g s[n][g] * P[m][n][g] (lm_head), P the exact int32 dot
+// product over 256-K (128-K) block g -- the W8A8 linear of "Qwen3.8-27B IQ8R
+// + DFlash2 -- radiance container" (rows "Weights" and "Activations"). The
+// u8 sub-scale changes every 256 of K, so each block's int32 result leaves
+// the tensor core and is promoted into an fp32 sum by the epilogue.
+//
+// Design (sm_100a, one CTA per SM, persistent over output tiles):
+//  - operands swapped so the per-row weight scales are per thread: the MMA's
+//    M side is a 128-row weight tile (TMEM lanes), its N side BM <= 256
+//    tokens (TMEM columns); D[n][m] = sum_k W[n][k] * Xq[m][k], both K-major;
+//  - warp 0 (one lane) loads 128-K slices of both operands with 2-D TMA
+//    (128-byte swizzle) into a 4-stage ring, weights evict-first, activations
+//    evict-last in L2 (they are reused by every weight tile);
+//  - warp 1 owns the tensor memory: it allocates two int32 accumulators of BM
+//    columns and one lane issues tcgen05.mma (4 per stage, K = 32 each),
+//    alternating accumulators per block and committing to mbarriers;
+//  - warps 2..17 are the epilogue: warp e covers TMEM lanes 32 (warp % 4) of
+//    column group e / 4. Per block each thread tcgen05.ld's its row's 16..64
+//    int32 sums, converts them exactly (|P| < 2^22: add the bits of 1.5*2^23
+//    and subtract it as a float) and FMAs them by its row's sub-scale into
+//    fp32 registers; at the tile's end it applies a[m] * s2[n] / 128 and
+//    stores bf16. Tiles walk the token dimension fastest, so concurrently
+//    running CTAs share weight tiles and the activations stay in L2.
+#pragma once
+
+#include <cuda.h>
+
+#include "iq8r_device.cuh"
+
+namespace iq8r {
+
+constexpr int kTcBN = 128;            // weight rows per tile (MMA M)
+constexpr int kTcMaxBM = 256;         // tokens per tile (MMA N)
+constexpr int kTcStageK = 128;        // K bytes per stage: one 128-byte swizzle row
+constexpr int kTcStages = 4;
+constexpr int kTcEpiWarps = 16;
+constexpr int kTcThreads = (2 + kTcEpiWarps) * 32;
+constexpr int kTcColsPerGroup = kTcMaxBM / 4;  // tokens per epilogue column group
+constexpr int kTcStageA = kTcBN * kTcStageK;                // 16 KB
+constexpr int kTcStageB = kTcMaxBM * kTcStageK;             // 32 KB
+constexpr int kTcStageBytes = kTcStageA + kTcStageB;        // 48 KB
+// stages, then barriers (13 x 8 B), the TMEM address, 2 x 256 activation
+// scales; plus 1 KB to align the stages to 1024 bytes
+constexpr int kTcSmemBytes = kTcStages * kTcStageBytes + 4096 + 1024;
+
+struct TcParams {
+  int64_t m;          // tokens
+  int64_t n;          // weight rows
+  int k;              // K (multiple of 256 for the trunk, 128 for lm_head)
+  int bm;             // tokens per tile: multiple of 16, 16..256
+  int fmt;            // 0 trunk, 1 lm_head
+  int rotated;
+  int64_t tiles_m;    // token tiles
+  int64_t tiles;      // total tiles
+  const float* xs;    // [m] activation scales
+  const uint8_t* sub; // [n][k/256]
+  const uint16_t* scale;  // [n] or [n][k/128]
+  uint16_t* y;        // [m][n], or nullptr in partials mode
+  int32_t* partials;  // [m][n][k/G] in partials mode
+  uint32_t tmem_cols; // columns allocated: 2 * bm rounded up to a power of two >= 32
+};
+
+// ------------------------------------------------------------ tcgen05 / TMA
+
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar,
+                                            uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3}], [%4], %5;" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_addr(bar)), "l"(policy)
+      : "memory");
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// Shared-memory matrix descriptor for a K-major operand stored as rows of
+// 128 bytes with the 128-byte swizzle (8-row atoms of 1024 bytes): start
+// address >> 4, leading offset 1 (unused for swizzled K-major), stride 1024 B
+// between 8-row groups, descriptor version 1, swizzle mode 2 (128 B).
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  return static_cast<uint64_t>((saddr >> 4) & 0x3FFFu) | (static_cast<uint64_t>(1) << 16) |
+         (static_cast<uint64_t>(1024 >> 4) << 32) | (static_cast<uint64_t>(1) << 46) |
+         (static_cast<uint64_t>(2) << 61);
+}
+
+// Instruction descriptor, kind::i8: s32 accumulator, signed int8 A and B,
+// both K-major, M = 128, N = bm.
+__device__ __forceinline__ uint32_t umma_idesc_i8(int bm) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(bm >> 3) << 17) | ((128u >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                        uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// The mbarrier arrives once every tcgen05 op this thread issued before has
+// completed (MMAs reading shared memory and writing TMEM).
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_addr(bar))
+               : "memory");
+}
+
+// 32 lanes x 16 consecutive 32-bit columns starting at taddr.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Exact int32 -> float for |v| < 2^22: the bits of 1.5 * 2^23 plus v are the
+// float 1.5 * 2^23 + v, and subtracting 1.5 * 2^23 is exact.
+__device__ __forceinline__ float small_int_to_float(uint32_t v) {
+  return __fsub_rn(__uint_as_float(v + 0x4B400000u), 12582912.0f);
+}
+
+// ------------------------------------------------------------------ kernel
+
+template <int FMT, bool PARTIALS>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
+                   const TcParams p) {
+  constexpr int G = FMT == 0 ? kGroupTrunk : kGroupHead;
+  constexpr int SPB = G / kTcStageK;  // stages per scale block: 2 (trunk) or 1 (lm_head)
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment for the swizzled TMA tiles
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* stage_base = smem;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);
+  uint64_t* empty = full + kTcStages;
+  uint64_t* acc_full = empty + kTcStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* mma_done = acc_empty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  float* sa = reinterpret_cast<float*>(tmem_slot + 4);  // [2][kTcMaxBM] activation scales per tile
+  __shared__ volatile int s_abort;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int K = p.k;
+  const int nkb = K / kTcStageK;       // stages per tile
+  const int ng = K / G;                // scale blocks per row
+  const int bm = p.bm;
+
+  if (threadIdx.x == 0) {
+    s_abort = 0;
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kTcEpiWarps);
+    }
+    mbar_init(mma_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_addr(tmem_slot)),
+                 "r"(p.tmem_cols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_x = l2_policy_evict_last();
+      const uint32_t tx = kTcStageA + bm * kTcStageK;
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
+        const int m0 = static_cast<int>((tile % p.tiles_m) * bm);
+        const int n0 = static_cast<int>((tile / p.tiles_m) * kTcBN);
+        for (int kb = 0; kb < nkb; ++kb, ++it) {
+          const int s = static_cast<int>(it % kTcStages);
+          const uint32_t use = it / kTcStages;
+          if (s_abort || (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1u, kDevErrTcEmpty))) {
+            s_abort = 1;
+            ok = false;
+            break;
+          }
+          uint8_t* st = stage_base + s * kTcStageBytes;
+          mbar_arrive_expect_tx(&full[s], tx);
+          tma_load_2d(st, &tmap_w, kb * kTcStageK, n0, &full[s], pol_w);
+          tma_load_2d(st + kTcStageA, &tmap_x, kb * kTcStageK, m0, &full[s], pol_x);
+        }
+      }
+      // never leave with a copy still landing in this CTA's shared memory
+      const uint32_t first = it > static_cast<uint32_t>(kTcStages) ? it - kTcStages : 0u;
+      for (uint32_t j = first; j < it; ++j)
+        if (!mbar_wait(&full[j % kTcStages], (j / kTcStages) & 1u, kDevErrTcDrain)) break;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      const uint32_t idesc = umma_idesc_i8(bm);
+      uint32_t it = 0;   // stages consumed
+      uint32_t blk = 0;  // accumulator blocks produced
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
+        for (int kb = 0; kb < nkb && ok; ++kb, ++it) {
+          const int buf = static_cast<int>(blk & 1u);
+          const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * bm);
+          if (kb % SPB == 0) {
+            // this accumulator must have been drained by the epilogue
+            const uint32_t use = blk >> 1;
+            if (s_abort || (use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1u, kDevErrTcAccEmpty))) {
+              s_abort = 1;
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+          }
+          const int s = static_cast<int>(it % kTcStages);
+          if (s_abort || !mbar_wait(&full[s], (it / kTcStages) & 1u, kDevErrTcFull)) {
+            s_abort = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_addr(stage_base + s * kTcStageBytes);
+          const uint32_t b_addr = a_addr + kTcStageA;
+#pragma unroll
+          for (int k = 0; k < kTcStageK / 32; ++k) {
+            // advancing K by 32 bytes inside the swizzle atom moves the start address
+            umma_i8(d_tmem, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k), idesc,
+                    (kb % SPB != 0 || k != 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);  // the stage can be refilled once these MMAs have read it
+          if (kb % SPB == SPB - 1) {
+            umma_commit(&acc_full[buf]);  // the block's int32 sums are complete
+            ++blk;
+          }
+        }
+      }
+      // every MMA issued here, complete or not, must be finished before the
+      // tensor memory is released
+      if (it > 0) {
+        umma_commit(mma_done);
+        mbar_wait(mma_done, 0u, kDevErrTcDrain);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int e = warp - 2;          // 0..15
+    const int q = e >> 2;            // column group: tokens [q * 64, q * 64 + 64) of the tile
+    const int lq = warp & 3;         // TMEM lane quarter this warp may access
+    const int cols = bm / 4;         // tokens per column group (bm is a multiple of 16)
+    const uint32_t lane_addr = static_cast<uint32_t>(lq * 32) << 16;
+    const float rot = p.rotated ? 0.0078125f : 1.0f;
+    uint32_t blk = 0;
+    int par = 0;
+    bool failed = false;
+    for (int64_t tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, par ^= 1) {
+      const int64_t m0 = (tile % p.tiles_m) * bm;
+      const int64_t n0 = (tile / p.tiles_m) * kTcBN;
+      const int64_t n = n0 + lq * 32 + lane;  // this thread's weight row
+      const bool nvalid = n < p.n;
+      // activation scales of the tile's tokens, shared by all epilogue warps
+      if (!PARTIALS) {
+        for (int i = e * 32 + lane; i < bm; i += kTcEpiWarps * 32)
+          sa[par * kTcMaxBM + i] = (m0 + i < p.m) ? p.xs[m0 + i] : 0.0f;
+      }
+      float s2f = 0.0f;
+      if (FMT == 0 && !PARTIALS && nvalid) s2f = bf16_bits_to_float(p.scale[n]);
+      float acc[kTcColsPerGroup];
+#pragma unroll
+      for (int j = 0; j < kTcColsPerGroup; ++j) acc[j] = 0.0f;
+      // the first block's scale, then one block ahead
+      float snext = 0.0f;
+      if (!PARTIALS && nvalid)
+        snext = FMT == 0 ? static_cast<float>(__ldg(p.sub + n * ng)) : bf16_bits_to_float(__ldg(p.scale + n * ng));
+      for (int g = 0; g < ng; ++g, ++blk) {
+        const float sg = snext;
+        if (!PARTIALS && nvalid && g + 1 < ng)
+          snext = FMT == 0 ? static_cast<float>(__ldg(p.sub + n * ng + g + 1))
+                           : bf16_bits_to_float(__ldg(p.scale + n * ng + g + 1));
+        const int buf = static_cast<int>(blk & 1u);
+        if (!failed) {
+          bool bad = s_abort != 0;
+          if (!bad) bad = !mbar_wait(&acc_full[buf], (blk >> 1) & 1u, kDevErrTcAccFull);
+          failed = !__all_sync(0xffffffffu, !bad);
+          if (failed && lane == 0) s_abort = 1;
+        }
+        tc_fence_after();
+        const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(buf * bm + q * cols);
+        if (!failed) {
+#pragma unroll
+          for (int c = 0; c < kTcColsPerGroup; c += 16) {
+            if (c < cols) {
+              uint32_t r[16];
+              tmem_ld16(tbase + c, r);
+              tmem_wait_ld();
+              if (PARTIALS) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  const int64_t m = m0 + q * cols + c + j;
+                  if (nvalid && m < p.m) p.partials[(m * p.n + n) * ng + g] = static_cast<int32_t>(r[j]);
+                }
+              } else {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) acc[c + j] = fmaf(small_int_to_float(r[j]), sg, acc[c + j]);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[buf]);
+      }
+      if (PARTIALS) continue;
+      // all epilogue warps have staged their part of sa before anyone reads it
+      named_barrier(1, kTcEpiWarps * 32);
+      if (!failed && nvalid) {
+        const float rs = (FMT == 0 ? s2f : 1.0f) * rot;
+#pragma unroll
+        for (int j = 0; j < kTcColsPerGroup; ++j) {
+          const int64_t m = m0 + q * cols + j;
+          if (j < cols && m < p.m)
+            p.y[m * p.n + n] = float_to_bf16_bits_rn(acc[j] * sa[par * kTcMaxBM + q * cols + j] * rs);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(p.tmem_cols)
+                 : "memory");
+  }
+}
+
+}  // namespace iq8r

@@ -39,6 +39,8 @@ constexpr int64_t kMaxGridRows = (int64_t(1) << 31) - 1;
 // iq8r_linear_bf16 fuses the activation quantiser into the GEMV up to this
 // many activation elements (M * K); beyond it two launches are cheaper.
 constexpr int64_t kFuseMaxElems = 16384;
+// Above this many tokens the automatic choice is the tensor-core GEMM.
+constexpr int64_t kGemvMaxM = 8;
 
 iq8r_status check_weight(const iq8r_weight* w, const char* fn) {
   if (!w) return fail(IQ8R_ERR_INVALID_ARG, "%s: weight is NULL", fn);
@@ -84,7 +86,7 @@ iq8r_status run_linear(const iq8r::LinearArgs& a, int32_t path, const char* fn, 
     if (!iq8r::gemm_tc_supported(a, &why)) return fail(IQ8R_ERR_UNSUPPORTED, "%s: %s", fn, why.c_str());
     use_tc = true;
   } else if (path == IQ8R_PATH_AUTO) {
-    use_tc = a.m > 8 && iq8r::gemm_tc_supported(a, nullptr);
+    use_tc = a.m > kGemvMaxM && iq8r::gemm_tc_supported(a, nullptr);
   }
   if (!use_tc && !iq8r::gemv_supported(a.k, &why)) {
     if (path == IQ8R_PATH_AUTO && iq8r::gemm_tc_supported(a, nullptr))

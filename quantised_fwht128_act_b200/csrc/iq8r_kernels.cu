@@ -5,7 +5,10 @@
 #include <atomic>
 #include <string>
 
+#include <cudaTypedefs.h>
+
 #include "act_quant.cuh"
+#include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "iq8r_device.cuh"
 #include "iq8r_internal.h"
@@ -208,12 +211,105 @@ bool gemv_supported(int64_t k, std::string* why) {
   return true;
 }
 
-bool gemm_tc_supported(const LinearArgs&, std::string* why) {
-  if (why) *why = "the tensor-core path is not available in this build";
-  return false;
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode_tiled = nullptr;
+std::atomic<int> g_encode_ready{0};
+
+// cuTensorMapEncodeTiled from the driver the runtime is using (no link to
+// libcuda needed).
+cudaError_t get_encode_tiled(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  if (g_encode_ready.load(std::memory_order_acquire) == 0) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || p == nullptr) return cudaErrorNotSupported;
+    g_encode_tiled = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    g_encode_ready.store(1, std::memory_order_release);
+  }
+  *fn = g_encode_tiled;
+  return cudaSuccess;
 }
 
-cudaError_t launch_gemm_tc(const LinearArgs&, cudaStream_t) { return cudaErrorNotSupported; }
+// Row-major int8 [rows][k] as 2-D TMA tiles of [box_rows][128 bytes], 128-byte
+// swizzle, out-of-range rows read as zeros.
+cudaError_t make_tmap_i8(CUtensorMap* map, const void* base, int64_t rows, int64_t k, int box_rows) {
+  PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  cudaError_t e = get_encode_tiled(&encode);
+  if (e != cudaSuccess) return e;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(k)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcStageK), static_cast<cuuint32_t>(box_rows)};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+template <int FMT, bool PARTIALS>
+cudaError_t launch_tc_t(const CUtensorMap& tw, const CUtensorMap& tx, const TcParams& p, int grid,
+                        cudaStream_t stream) {
+  auto kernel = gemm_tc_kernel<FMT, PARTIALS>;
+  static std::atomic<int> configured[kMaxDevices];
+  cudaError_t e = ensure_smem(kernel, kTcSmemBytes, configured);
+  if (e != cudaSuccess) return e;
+  kernel<<<grid, kTcThreads, kTcSmemBytes, stream>>>(tw, tx, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool gemm_tc_supported(const LinearArgs& a, std::string* why) {
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) {
+    if (why) *why = "cannot query the current device";
+    return false;
+  }
+  if (d.smem_optin < kTcSmemBytes + 1024) {
+    if (why) *why = "not enough shared memory per block for the tensor-core kernel";
+    return false;
+  }
+  if (a.k % kTcStageK) {
+    if (why) *why = "K must be a multiple of 128";
+    return false;
+  }
+  return true;
+}
+
+cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream) {
+  if (a.m == 0 || a.n == 0) return cudaSuccess;
+  DeviceInfo d;
+  cudaError_t e = device_info(&d);
+  if (e != cudaSuccess) return e;
+  TcParams p{};
+  p.m = a.m;
+  p.n = a.n;
+  p.k = static_cast<int>(a.k);
+  p.bm = a.m >= kTcMaxBM ? kTcMaxBM : static_cast<int>((a.m + 15) / 16 * 16);
+  p.fmt = a.fmt;
+  p.rotated = a.rotated;
+  p.tiles_m = (a.m + p.bm - 1) / p.bm;
+  p.tiles = p.tiles_m * ((a.n + kTcBN - 1) / kTcBN);
+  p.xs = a.xs;
+  p.sub = a.sub;
+  p.scale = a.scale;
+  p.y = a.y;
+  p.partials = a.partials;
+  uint32_t cols = 32;
+  while (cols < static_cast<uint32_t>(2 * p.bm)) cols <<= 1;
+  p.tmem_cols = cols;
+  CUtensorMap tw, tx;
+  e = make_tmap_i8(&tw, a.codes, a.n, a.k, kTcBN);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_i8(&tx, a.xq, a.m, a.k, p.bm);
+  if (e != cudaSuccess) return e;
+  const int grid = static_cast<int>(std::min<int64_t>(d.num_sms, p.tiles));
+  const bool part = a.partials != nullptr;
+  if (a.fmt == 0) return part ? launch_tc_t<0, true>(tw, tx, p, grid, stream) : launch_tc_t<0, false>(tw, tx, p, grid, stream);
+  return part ? launch_tc_t<1, true>(tw, tx, p, grid, stream) : launch_tc_t<1, false>(tw, tx, p, grid, stream);
+}
 
 namespace {
 

@@ -312,3 +312,43 @@ def test_linear_bf16_large_m_stages_codes():
     st = iq8r.lib().iq8r_linear_bf16(dev_bf16(x).data_ptr(), x.shape[0], ctypes.byref(w), y.data_ptr(), None, None,
                                       torch.cuda.current_stream().cuda_stream)
     assert st == iq8r.IQ8R_ERR_INVALID_ARG
+
+
+# --------------------------------------------------- tensor-core path (TC)
+
+TC_SHAPES = [(16, 128, 512), (200, 300, 768), (257, 129, 256), (33, 1000, 2304), (512, 256, 5120)]
+
+
+@pytest.mark.parametrize("m,n,k", TC_SHAPES)
+def test_tc_partials_bit_exact(m, n, k):
+    """tcgen05 kind::i8: per-256-K int32 sums equal the oracle's exactly
+    (token and weight tile tails, odd block counts, several tiles)."""
+    x, _, _, (codes, _, _), W = case("decode", m=m, n=n, k=k, seed=71 + m + n + k)
+    xq, _ = oracle.act_quant(x)
+    got = gpu_partials(x, W, path=iq8r.IQ8R_PATH_TC)
+    assert np.array_equal(got, oracle.partials(xq, codes, 256))
+
+
+@pytest.mark.parametrize("m,n,k", TC_SHAPES)
+def test_tc_linear_within_tolerance(m, n, k):
+    x, _, fmt, packed, W = case("decode", m=m, n=n, k=k, seed=71 + m + n + k)
+    y64 = oracle_linear(x, fmt, packed)
+    y = gpu_linear(x, W, path=iq8r.IQ8R_PATH_TC)
+    st = check_output(y, y64, oracle.linear_bf16(y64))
+    assert st["bit_equal_frac"] > 0.98
+
+
+def test_tc_lm_head_format():
+    x, _, fmt, packed, W = case("lm_head8", m=40, n=256, k=640, seed=72)
+    codes = packed[0]
+    xq, _ = oracle.act_quant(x)
+    assert np.array_equal(gpu_partials(x, W, path=iq8r.IQ8R_PATH_TC), oracle.partials(xq, codes, 128))
+    y64 = oracle_linear(x, fmt, packed)
+    check_output(gpu_linear(x, W, path=iq8r.IQ8R_PATH_TC), y64, oracle.linear_bf16(y64))
+
+
+def test_tc_and_gemv_agree_on_partials():
+    x, _, _, _, W = case("decode", m=24, n=512, k=1024, seed=73)
+    a = gpu_partials(x, W, path=iq8r.IQ8R_PATH_TC)
+    b = gpu_partials(x, W, path=iq8r.IQ8R_PATH_GEMV)
+    assert np.array_equal(a, b)
