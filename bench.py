@@ -2,9 +2,13 @@
 """Benchmark of the IQ8R rotated W8A8 linear (libiq8r) on B200.
 
 A step is one pass of the whole hot path over one batch: rotate + int8
-quantise the activations (iq8r_rotate_quant_act), then the int8 linear with
-its fused scale epilogue (iq8r_linear). The default workload is the decode
-GEMV (M=1, K=5120, N=17408, trunk format); --config picks another.
+quantise the activations, then the int8 linear with its fused scale
+epilogue. For M <= 8 that is one launch (iq8r_linear_bf16: the GEMV rotates
+and quantises x itself); above, iq8r_rotate_quant_act then the tcgen05
+tensor-core GEMM (iq8r_linear). The default workload is the decode GEMV
+(M=1, K=5120, N=17408, trunk format), reported in HBM GB/s, with a
+"prefill" object (M=8192, int8 TOPS) in the same line; --config picks
+another workload.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config decode]
     python bench.py --impl reference ...   # the CPU oracle, same metric
@@ -227,7 +231,7 @@ def run_ours(args, rank, world, local_rank):
     xsc = [torch.empty((m,), dtype=torch.float32, device=dev) for _ in range(R)]
     y = [torch.empty((m, n), dtype=torch.bfloat16, device=dev) for _ in range(R)]
     fused = m <= 8  # one launch: the GEMV rotates and quantises x itself
-    launches_per_step = 1 if fused else 1 + (m + 7) // 8  # else act + GEMV groups of 8 tokens
+    launches_per_step = 1 if fused else 2  # else the activation kernel + the tensor-core GEMM
 
     def step(j):
         r = j % R
@@ -353,7 +357,9 @@ def run_ours(args, rank, world, local_rank):
             t = torch.tensor([e_ms], device=dev)
             torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
             e_ms = float(t.item())
-        e2e = {"value": world * step_bytes(m, k, n, fmt) * Ke / (e_ms * 1e-3) / 1e9, "unit": "GB/s",
+        e_val = (world * 2.0 * m * n * k * Ke / (e_ms * 1e-3) / 1e12 if m > 8
+                 else world * step_bytes(m, k, n, fmt) * Ke / (e_ms * 1e-3) / 1e9)
+        e2e = {"value": e_val, "unit": "TOPS" if m > 8 else "GB/s",
                "h2d_bytes_per_step": 2 * m * k, "d2h_bytes_per_step": 2 * m * n, "steps": Ke,
                "ms_per_step": e_ms / Ke, "how": "eager public-API calls on one stream, pinned host buffers"}
 
@@ -371,21 +377,33 @@ def run_ours(args, rank, world, local_rank):
                 "traffic": recorded_traffic("gemv_kernel", args.config, kern_files),
                 "algorithmic_bytes_per_launch": lin_b, "avg_launch_ms": lin_avg_ms}
     else:
+        # a dense int8 contraction on the tensor cores: its roofline is the int8
+        # tensor peak, the measured bf16 peak times the nominal int8/bf16 ratio
         ops = 2.0 * m * n * k
-        achieved_b = lin_b / (lin_avg_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "kernel": "gemv_kernel (token groups of 8)", "achieved": achieved_b, "peak": hbm,
-                "unit": "GB/s", "frac": achieved_b / hbm,
-                "int8_tops": ops / (lin_avg_ms * 1e-3) / 1e12,
-                "traffic": recorded_traffic("gemv_kernel", args.config, kern_files),
-                "algorithmic_bytes_per_launch": lin_b, "avg_launch_ms": lin_avg_ms}
+        peak_i8 = bf16_tf * INT8_OVER_BF16
+        achieved_t = ops / (lin_avg_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "kernel": "gemm_tc_kernel (tcgen05 kind::i8)", "achieved": achieved_t,
+                "peak": peak_i8, "unit": "TOPS", "frac": achieved_t / peak_i8,
+                "peak_source": (f"{peak_src} cuBLAS bf16 {bf16_tf:.1f} TFLOP/s (MEASURED_PEAKS.json bf16_tflops) "
+                                f"x {INT8_OVER_BF16:g} (nominal dense int8/bf16)"),
+                "frac_of_datasheet_4500": achieved_t / 4500.0,
+                "hbm_gbs": lin_b / (lin_avg_ms * 1e-3) / 1e9,
+                "traffic": recorded_traffic("gemm_tc_kernel", args.config, ["gemm_tc.cuh", "iq8r_device.cuh"]),
+                "algorithmic_ops_per_launch": ops, "algorithmic_bytes_per_launch": lin_b,
+                "avg_launch_ms": lin_avg_ms}
     if not fused:
         roof["act_kernel"] = {"avg_launch_ms": act_avg_ms, "bytes": act_bytes(m, k),
-                              "achieved_gbs": act_bytes(m, k) / (act_avg_ms * 1e-3) / 1e9}
+                              "achieved_gbs": act_bytes(m, k) / (act_avg_ms * 1e-3) / 1e9,
+                              "frac_of_hbm": act_bytes(m, k) / (act_avg_ms * 1e-3) / 1e9 / hbm}
 
     value = world * step_bytes(m, k, n, fmt) * K / (elapsed_ms * 1e-3) / 1e9
+    unit = "GB/s"
+    if m > 8:  # prefill-like steps are reported in int8 TOPS
+        value = world * 2.0 * m * n * k * K / (elapsed_ms * 1e-3) / 1e12
+        unit = "TOPS"
     clocks = sampler.summary(t_start_wall, t_end_wall)
     out = {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": elapsed_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8", "data": "synthetic",
         "config": {"workload": args.config, "m": m, "k": k, "n": n, "format": fmt, "rotated": True,
@@ -464,7 +482,7 @@ def run_reference(args, rank, world):
     value, sample, reps, s_per = run_oracle(args.config, budget, steps=K)
     cores = blas_threads()
     return {
-        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": s_per * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8", "data": "synthetic", "impl": "reference",
         "config": {"workload": args.config, "m": m, "k": k, "n": n, "format": fmt, "rotated": True},
@@ -484,6 +502,7 @@ def main(argv=None):
     ap.add_argument("--config", choices=sorted(CONFIGS), default="decode")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the prefill TOPS line of the decode run")
     ap.add_argument("--cpu-budget-s", type=float, default=15.0)
     args = ap.parse_args(argv)
     if args.steps is None:
@@ -510,6 +529,16 @@ def main(argv=None):
                                              device_id=torch.device("cuda", local_rank))
     try:
         out = run_ours(args, rank, world, local_rank)
+        if args.config == "decode" and not args.no_prefill:
+            # the metric's second half: prefill int8 TOPS on the tensor cores
+            pargs = argparse.Namespace(**vars(args))
+            pargs.config = "prefill"
+            pargs.steps = CONFIGS["prefill"][4]
+            pargs.warmup = min(args.warmup, 5)
+            pargs.no_e2e = True
+            pre = run_ours(pargs, rank, world, local_rank)
+            out["prefill"] = {k_: pre[k_] for k_ in ("value", "unit", "steps", "warmup", "ms_per_step", "config",
+                                                       "roofline", "gpu_launches", "clocks")}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             value, sample, reps, _ = run_oracle(args.config, args.cpu_budget_s)
             out["cpu_baseline"] = {"value": value, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",

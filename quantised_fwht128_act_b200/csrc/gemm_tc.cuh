@@ -17,13 +17,15 @@
 //    evict-last in L2 (they are reused by every weight tile);
 //  - warp 1 owns the tensor memory: it allocates two int32 accumulators of BM
 //    columns and one lane issues tcgen05.mma (4 per stage, K = 32 each),
-//    alternating accumulators per block and committing to mbarriers;
-//  - warps 2..17 are the epilogue: warp e covers TMEM lanes 32 (warp % 4) of
-//    column group e / 4. Per block each thread tcgen05.ld's its row's 16..64
-//    int32 sums, converts them exactly (|P| < 2^22: add the bits of 1.5*2^23
-//    and subtract it as a float) and FMAs them by its row's sub-scale into
-//    fp32 registers; at the tile's end it applies a[m] * s2[n] / 128 and
-//    stores bf16. Tiles walk the token dimension fastest, so concurrently
+//    always accumulating, alternating accumulators per block and
+//    committing to mbarriers;
+//  - warps 2..9 are the epilogue: warp e covers TMEM lanes 32 (warp % 4) of
+//    column group e / 4 (half the tile's tokens). The accumulators start each block at the bits of
+//    1.5 * 2^23, so the int32 sums read back (tcgen05.ld) are the floats
+//    1.5 * 2^23 + P: one packed f32x2 subtract makes P exact and one packed
+//    f32x2 FMA adds P times the row's sub-scale into fp32 registers; the
+//    epilogue writes the bias back (tcgen05.st) before releasing the buffer.
+//    At the tile's end it applies a[m] * s2[n] / 128 and stores bf16. Tiles walk the token dimension fastest, so concurrently
 //    running CTAs share weight tiles and the activations stay in L2.
 #pragma once
 
@@ -37,9 +39,10 @@ constexpr int kTcBN = 128;            // weight rows per tile (MMA M)
 constexpr int kTcMaxBM = 256;         // tokens per tile (MMA N)
 constexpr int kTcStageK = 128;        // K bytes per stage: one 128-byte swizzle row
 constexpr int kTcStages = 4;
-constexpr int kTcEpiWarps = 16;
+constexpr int kTcEpiWarps = 8;                 // 4 TMEM lane quarters x kTcGroups column groups
+constexpr int kTcGroups = kTcEpiWarps / 4;
 constexpr int kTcThreads = (2 + kTcEpiWarps) * 32;
-constexpr int kTcColsPerGroup = kTcMaxBM / 4;  // tokens per epilogue column group
+constexpr int kTcColsPerGroup = kTcMaxBM / kTcGroups;  // tokens per epilogue column group
 constexpr int kTcStageA = kTcBN * kTcStageK;                // 16 KB
 constexpr int kTcStageB = kTcMaxBM * kTcStageK;             // 32 KB
 constexpr int kTcStageBytes = kTcStageA + kTcStageB;        // 48 KB
@@ -129,10 +132,47 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// Exact int32 -> float for |v| < 2^22: the bits of 1.5 * 2^23 plus v are the
-// float 1.5 * 2^23 + v, and subtracting 1.5 * 2^23 is exact.
-__device__ __forceinline__ float small_int_to_float(uint32_t v) {
-  return __fsub_rn(__uint_as_float(v + 0x4B400000u), 12582912.0f);
+// 32 lanes x 16 consecutive 32-bit columns, all set to v.
+__device__ __forceinline__ void tmem_st16_fill(uint32_t taddr, uint32_t v) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, %1, "
+      "%1};" ::"r"(taddr),
+      "r"(v)
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// The accumulators start every block at the bits of 1.5 * 2^23 (as an int32)
+// instead of 0, so the MMA's exact int32 sum P (|P| < 2^22) lands in the
+// float 1.5 * 2^23 + P, and subtracting 1.5 * 2^23 recovers P exactly.
+constexpr uint32_t kTcBiasBits = 0x4B400000u;
+constexpr float kTcBias = 12582912.0f;
+
+// Two fp32 lanes in one 64-bit register: Blackwell's packed f32x2 add and
+// fma do both halves in one instruction, each rounded like the scalar op.
+__device__ __forceinline__ uint64_t u2_pack(uint32_t lo, uint32_t hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "r"(lo), "r"(hi));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_splat(float v) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %1};" : "=l"(r) : "f"(v));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
 }
 
 // ------------------------------------------------------------------ kernel
@@ -230,8 +270,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * bm);
           if (kb % SPB == 0) {
             // this accumulator must have been drained by the epilogue
+            // drained by the epilogue and reset to the bias (seeded once at start)
             const uint32_t use = blk >> 1;
-            if (s_abort || (use > 0 && !mbar_wait(&acc_empty[buf], (use - 1) & 1u, kDevErrTcAccEmpty))) {
+            if (s_abort || !mbar_wait(&acc_empty[buf], use & 1u, kDevErrTcAccEmpty)) {
               s_abort = 1;
               ok = false;
               break;
@@ -250,8 +291,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
           for (int k = 0; k < kTcStageK / 32; ++k) {
             // advancing K by 32 bytes inside the swizzle atom moves the start address
-            umma_i8(d_tmem, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k), idesc,
-                    (kb % SPB != 0 || k != 0) ? 1u : 0u);
+            umma_i8(d_tmem, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k), idesc, 1u);
           }
           umma_commit(&empty[s]);  // the stage can be refilled once these MMAs have read it
           if (kb % SPB == SPB - 1) {
@@ -269,12 +309,25 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int e = warp - 2;          // 0..15
-    const int q = e >> 2;            // column group: tokens [q * 64, q * 64 + 64) of the tile
+    const int e = warp - 2;          // 0 .. kTcEpiWarps - 1
+    const int q = e >> 2;            // column group: tokens [q * cols, (q + 1) * cols) of the tile
     const int lq = warp & 3;         // TMEM lane quarter this warp may access
-    const int cols = bm / 4;         // tokens per column group (bm is a multiple of 16)
+    const int cols = bm / kTcGroups; // tokens per column group (a multiple of 16 when bm is of 32)
     const uint32_t lane_addr = static_cast<uint32_t>(lq * 32) << 16;
     const float rot = p.rotated ? 0.0078125f : 1.0f;
+    // seed both accumulators with the bias (this warp's lanes and columns)
+    for (int b = 0; b < 2; ++b) {
+      const uint32_t t0 = tmem_base + lane_addr + static_cast<uint32_t>(b * bm + q * cols);
+      for (int c = 0; c < cols; c += 16) tmem_st16_fill(t0 + c, kTcBiasBits);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&acc_empty[0]);
+      mbar_arrive(&acc_empty[1]);
+    }
+    const uint64_t neg_bias = f2_splat(-kTcBias);
     uint32_t blk = 0;
     int par = 0;
     bool failed = false;
@@ -290,15 +343,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       float s2f = 0.0f;
       if (FMT == 0 && !PARTIALS && nvalid) s2f = bf16_bits_to_float(p.scale[n]);
-      float acc[kTcColsPerGroup];
+      uint64_t acc[kTcColsPerGroup / 2];  // fp32 pairs
 #pragma unroll
-      for (int j = 0; j < kTcColsPerGroup; ++j) acc[j] = 0.0f;
+      for (int j = 0; j < kTcColsPerGroup / 2; ++j) acc[j] = 0ull;
       // the first block's scale, then one block ahead
       float snext = 0.0f;
       if (!PARTIALS && nvalid)
         snext = FMT == 0 ? static_cast<float>(__ldg(p.sub + n * ng)) : bf16_bits_to_float(__ldg(p.scale + n * ng));
       for (int g = 0; g < ng; ++g, ++blk) {
-        const float sg = snext;
+        const uint64_t sg = f2_splat(snext);
         if (!PARTIALS && nvalid && g + 1 < ng)
           snext = FMT == 0 ? static_cast<float>(__ldg(p.sub + n * ng + g + 1))
                            : bf16_bits_to_float(__ldg(p.scale + n * ng + g + 1));
@@ -311,26 +364,46 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         tc_fence_after();
         const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(buf * bm + q * cols);
-        if (!failed) {
+        // with few columns per thread, chunk c + 1 loads while chunk c is
+        // converted and summed; with many, registers are kept for the sums
+        constexpr bool kPipe = kTcColsPerGroup <= 64;
+        uint32_t rn[16];
+        if (kPipe && !failed) {
+          tmem_ld16(tbase, rn);
+          tmem_wait_ld();
+        }
 #pragma unroll
-          for (int c = 0; c < kTcColsPerGroup; c += 16) {
-            if (c < cols) {
-              uint32_t r[16];
+        for (int c = 0; c < kTcColsPerGroup; c += 16) {
+          if (c < cols) {
+            uint32_t r[16];
+            if (kPipe) {
+#pragma unroll
+              for (int j = 0; j < 16; ++j) r[j] = rn[j];
+              if (!failed && c + 16 < cols) tmem_ld16(tbase + c + 16, rn);
+            } else if (!failed) {
               tmem_ld16(tbase + c, r);
               tmem_wait_ld();
-              if (PARTIALS) {
+            }
+            tmem_st16_fill(tbase + c, kTcBiasBits);  // reset for the block after next
+            if (failed) continue;
+            if (PARTIALS) {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                  const int64_t m = m0 + q * cols + c + j;
-                  if (nvalid && m < p.m) p.partials[(m * p.n + n) * ng + g] = static_cast<int32_t>(r[j]);
-                }
-              } else {
+              for (int j = 0; j < 16; ++j) {
+                const int64_t m = m0 + q * cols + c + j;
+                if (nvalid && m < p.m)
+                  p.partials[(m * p.n + n) * ng + g] = static_cast<int32_t>(r[j] - kTcBiasBits);
+              }
+            } else {
 #pragma unroll
-                for (int j = 0; j < 16; ++j) acc[c + j] = fmaf(small_int_to_float(r[j]), sg, acc[c + j]);
+              for (int j = 0; j < 16; j += 2) {
+                const uint64_t v = f2_add(u2_pack(r[j], r[j + 1]), neg_bias);  // exact: P
+                acc[(c + j) / 2] = f2_fma(v, sg, acc[(c + j) / 2]);
               }
             }
+            if (kPipe && c + 16 < cols) tmem_wait_ld();
           }
         }
+        tmem_wait_st();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
@@ -341,10 +414,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       if (!failed && nvalid) {
         const float rs = (FMT == 0 ? s2f : 1.0f) * rot;
 #pragma unroll
-        for (int j = 0; j < kTcColsPerGroup; ++j) {
+        for (int j = 0; j < kTcColsPerGroup; j += 2) {
+          float a0, a1;
+          f2_unpack(acc[j / 2], a0, a1);
           const int64_t m = m0 + q * cols + j;
           if (j < cols && m < p.m)
-            p.y[m * p.n + n] = float_to_bf16_bits_rn(acc[j] * sa[par * kTcMaxBM + q * cols + j] * rs);
+            p.y[m * p.n + n] = float_to_bf16_bits_rn(a0 * sa[par * kTcMaxBM + q * cols + j] * rs);
+          if (j + 1 < cols && m + 1 < p.m)
+            p.y[(m + 1) * p.n + n] = float_to_bf16_bits_rn(a1 * sa[par * kTcMaxBM + q * cols + j + 1] * rs);
         }
       }
     }

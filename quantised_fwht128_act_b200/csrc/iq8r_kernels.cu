@@ -287,7 +287,9 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream) {
   p.m = a.m;
   p.n = a.n;
   p.k = static_cast<int>(a.k);
-  p.bm = a.m >= kTcMaxBM ? kTcMaxBM : static_cast<int>((a.m + 15) / 16 * 16);
+  // tokens per tile: each of the kTcGroups column groups needs a multiple of 16
+  constexpr int64_t kBmStep = 16 * kTcGroups;
+  p.bm = a.m >= kTcMaxBM ? kTcMaxBM : static_cast<int>((a.m + kBmStep - 1) / kBmStep * kBmStep);
   p.fmt = a.fmt;
   p.rotated = a.rotated;
   p.tiles_m = (a.m + p.bm - 1) / p.bm;
