@@ -13,8 +13,9 @@
 //    M side is a 128-row weight tile (TMEM lanes), its N side BM <= 256
 //    tokens (TMEM columns); D[n][m] = sum_k W[n][k] * Xq[m][k], both K-major;
 //  - warp 0 (one lane) loads 128-K slices of both operands with 2-D TMA
-//    (128-byte swizzle) into a 4-stage ring, weights evict-first, activations
-//    evict-last in L2 (they are reused by every weight tile);
+//    (128-byte swizzle) into a 4-stage ring, activations evict-last in L2
+//    (they are reused by every weight tile); the output is stored streaming
+//    (evict-first) so it does not push out weight tiles other CTAs still read;
 //  - warp 1 owns the tensor memory: it allocates two int32 accumulators of BM
 //    columns and one lane issues tcgen05.mma (4 per stage, K = 32 each),
 //    always accumulating, alternating accumulators per block and
@@ -81,6 +82,12 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, i
 __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   uint64_t pol;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ uint64_t l2_policy_evict_normal() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
 
@@ -230,7 +237,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_first();
+      const uint64_t pol_w = l2_policy_evict_normal();
       const uint64_t pol_x = l2_policy_evict_last();
       const uint32_t tx = kTcStageA + bm * kTcStageK;
       uint32_t it = 0;
@@ -419,9 +426,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           f2_unpack(acc[j / 2], a0, a1);
           const int64_t m = m0 + q * cols + j;
           if (j < cols && m < p.m)
-            p.y[m * p.n + n] = float_to_bf16_bits_rn(a0 * sa[par * kTcMaxBM + q * cols + j] * rs);
+            __stcs(p.y + m * p.n + n, float_to_bf16_bits_rn(a0 * sa[par * kTcMaxBM + q * cols + j] * rs));
           if (j + 1 < cols && m + 1 < p.m)
-            p.y[(m + 1) * p.n + n] = float_to_bf16_bits_rn(a1 * sa[par * kTcMaxBM + q * cols + j + 1] * rs);
+            __stcs(p.y + (m + 1) * p.n + n, float_to_bf16_bits_rn(a1 * sa[par * kTcMaxBM + q * cols + j + 1] * rs));
         }
       }
     }

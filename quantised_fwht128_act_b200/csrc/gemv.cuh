@@ -250,10 +250,7 @@ __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
     for (int i = threadIdx.x; i < n16; i += blockDim.x) pad[i] = make_int4(0, 0, 0, 0);
   }
   __syncthreads();
-  if (!FUSED && threadIdx.x == 0) {
-    mbar_arrive_expect_tx(actbar, static_cast<uint32_t>(M * K));
-    bulk_g2s_default(act, a.xq, static_cast<uint32_t>(M * K), actbar);
-  }
+  pdl_launch_dependents();
   const uint64_t pol = l2_policy_evict_first();
 
   // ---- issuing (lane 0): claim work, fill stage buffer `b`
@@ -320,10 +317,17 @@ __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
     }
   };
 
+  // the first stages hold only weights, which no earlier kernel writes: they
+  // stream while the previous kernel on the stream finishes
   for (int b = 0; b < p.depth; ++b) issue(b);
+  pdl_wait();
+  if (!FUSED && threadIdx.x == 0) {
+    mbar_arrive_expect_tx(actbar, static_cast<uint32_t>(M * K));
+    bulk_g2s_default(act, a.xq, static_cast<uint32_t>(M * K), actbar);
+  }
 
   // activation codes: computed here (fused) while the first stages stream,
-  // or already on their way by bulk copy
+  // or on their way by bulk copy
   float xscale[MT];
   bool failed = false;  // warp-uniform: a wait ran out; stop computing
   if (FUSED) {

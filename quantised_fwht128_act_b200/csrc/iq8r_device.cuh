@@ -35,6 +35,16 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
 }
 
 // Make barrier initialisation visible to the async (bulk copy) proxy.
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialisation may start while the stream's previous kernel is finishing;
+// pdl_wait() blocks until that kernel has completed and its writes are
+// visible, so everything before it may only read data no earlier kernel
+// writes (the weights). pdl_launch_dependents() lets the next kernel start
+// once every CTA of this one has issued it or exited. Both are no-ops for a
+// plain launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void fence_barrier_init() {
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -92,8 +92,20 @@ cudaError_t launch_gemv_t(const LinearArgs& a, const GemvPlan& p, const DeviceIn
   if (e != cudaSuccess) return e;
   const int64_t tiles = (a.n + p.rt - 1) / p.rt;
   const int64_t grid = std::min<int64_t>(d.num_sms, tiles);
-  kernel<<<static_cast<unsigned>(grid), p.warps * 32, p.smem, stream>>>(a, p, tiles / grid, tiles % grid);
-  return cudaGetLastError();
+  // programmatic dependent launch: the kernel's first weight stages stream
+  // while the stream's previous kernel drains (the kernel waits for it before
+  // touching activations or outputs)
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(p.warps * 32);
+  cfg.dynamicSmemBytes = static_cast<size_t>(p.smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a, p, tiles / grid, tiles % grid);
 }
 
 template <int FMT, int MODE>
