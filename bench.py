@@ -81,12 +81,43 @@ def fused_bytes(m, k, n, fmt):
     return linear_bytes(m, k, n, fmt) - m * k - 4 * m + 2 * m * k
 
 
-def step_bytes(m, k, n, fmt):
-    """Algorithmic bytes of one step: the fused layer for M <= 8, else the
-    activation kernel plus the linear."""
-    if m <= 8:
+def step_bytes(m, k, n, fmt, fused=None):
+    """Algorithmic bytes of one step: the fused layer (one launch, M <= 8),
+    else the activation kernel plus the linear."""
+    if fused is None:
+        fused = m <= 8
+    if fused:
         return fused_bytes(m, k, n, fmt)
     return act_bytes(m, k) + linear_bytes(m, k, n, fmt)
+
+
+def max_over_ranks(ms, world, device):
+    """The slowest rank's time: every rank takes the same all-reduce (MAX),
+    so the job's throughput is all ranks' work over this time."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([float(ms)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(units_per_rank, world, ms_max):
+    """Whole-job throughput: the units all ranks processed per second of the
+    slowest rank."""
+    return world * units_per_rank / (ms_max * 1e-3)
+
+
+def is_hbm_bound(m, k, n, fmt, fused=None):
+    """The step's bound: HBM below the ridge point (int8 ops per algorithmic
+    byte at which the int8 tensor peak and the HBM peak take equal time),
+    the tensor cores above it. Decode and verify steps are HBM-bound and are
+    reported in GB/s; prefill is tensor-bound and reported in int8 TOPS."""
+    if fused is None:
+        fused = m <= 8
+    hbm, bf16_tf, _ = peaks()
+    lin_b = fused_bytes(m, k, n, fmt) if fused else linear_bytes(m, k, n, fmt)
+    return 2.0 * m * n * k / lin_b < bf16_tf * INT8_OVER_BF16 * 1e12 / (hbm * 1e9)
 
 
 # ------------------------------------------------------------------ peaks
@@ -230,7 +261,12 @@ def run_ours(args, rank, world, local_rank):
     xq = [torch.empty((m, k), dtype=torch.int8, device=dev) for _ in range(R)]
     xsc = [torch.empty((m,), dtype=torch.float32, device=dev) for _ in range(R)]
     y = [torch.empty((m, n), dtype=torch.bfloat16, device=dev) for _ in range(R)]
-    fused = m <= 8  # one launch: the GEMV rotates and quantises x itself
+    path = {"auto": iq8r.IQ8R_PATH_AUTO, "gemv": iq8r.IQ8R_PATH_GEMV, "tc": iq8r.IQ8R_PATH_TC}[args.path]
+    fused = m <= 8 and args.path == "auto"  # one launch: the GEMV rotates and quantises x itself
+
+    def linear(r):
+        iq8r.iq8r_linear_ex(xq[r], xsc[r], weights[r], y[r], path=path)
+
     launches_per_step = 1 if fused else 2  # else the activation kernel + the tensor-core GEMM
 
     def step(j):
@@ -239,7 +275,7 @@ def run_ours(args, rank, world, local_rank):
             iq8r.iq8r_linear_bf16(x_dev[r], weights[r], y[r])
         else:
             iq8r.iq8r_rotate_quant_act(x_dev[r], True, xq[r], xsc[r])
-            iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
+            linear(r)
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
@@ -270,7 +306,7 @@ def run_ours(args, rank, world, local_rank):
                 evs[j][0].record()
                 iq8r.iq8r_rotate_quant_act(x_dev[r], True, xq[r], xsc[r])
                 evs[j][1].record()
-                iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
+                linear(r)
                 evs[j][2].record()
         return g, evs
 
@@ -316,10 +352,7 @@ def run_ours(args, rank, world, local_rank):
         evs = ev_main if ev_main is not None else ev_tail
         act_ms = [e[0].elapsed_time(e[1]) for e in evs]
         lin_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, world, dev)
     del g_main, g_tail
 
     # end to end through the public API: pinned H2D of x, the two calls,
@@ -338,7 +371,7 @@ def run_ours(args, rank, world, local_rank):
                     iq8r.iq8r_linear_bf16(xin[r], weights[r], y[r])
                 else:
                     iq8r.iq8r_rotate_quant_act(xin[r], True, xq[r], xsc[r])
-                    iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
+                    linear(r)
                 yh[r].copy_(y[r], non_blocking=True)
         stream.synchronize()
         if world > 1:
@@ -355,18 +388,16 @@ def run_ours(args, rank, world, local_rank):
                     iq8r.iq8r_linear_bf16(xin[r], weights[r], y[r])
                 else:
                     iq8r.iq8r_rotate_quant_act(xin[r], True, xq[r], xsc[r])
-                    iq8r.iq8r_linear(xq[r], xsc[r], weights[r], y[r])
+                    linear(r)
                 yh[r].copy_(y[r], non_blocking=True)
             s1.record()
         stream.synchronize()
         e_ms = s0.elapsed_time(s1)
-        if world > 1:
-            t = torch.tensor([e_ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e_val = (world * 2.0 * m * n * k * Ke / (e_ms * 1e-3) / 1e12 if m > 8
-                 else world * step_bytes(m, k, n, fmt) * Ke / (e_ms * 1e-3) / 1e9)
-        e2e = {"value": e_val, "unit": "TOPS" if m > 8 else "GB/s",
+        e_ms = max_over_ranks(e_ms, world, dev)
+        e_hbm = is_hbm_bound(m, k, n, fmt, fused)
+        e_val = (job_value(step_bytes(m, k, n, fmt, fused) * Ke, world, e_ms) / 1e9 if e_hbm
+                 else job_value(2.0 * m * n * k * Ke, world, e_ms) / 1e12)
+        e2e = {"value": e_val, "unit": "GB/s" if e_hbm else "TOPS",
                "h2d_bytes_per_step": 2 * m * k, "d2h_bytes_per_step": 2 * m * n, "steps": Ke,
                "ms_per_step": e_ms / Ke, "how": "eager public-API calls on one stream, pinned host buffers"}
 
@@ -374,28 +405,36 @@ def run_ours(args, rank, world, local_rank):
     lin_avg_ms = float(np.mean(lin_ms))
     act_avg_ms = float(np.mean(act_ms))
     lin_b = fused_bytes(m, k, n, fmt) if fused else linear_bytes(m, k, n, fmt)
-    kern_files = ["gemv.cuh", "act_quant.cuh", "iq8r_device.cuh"]
-    if m <= 8:
+    ops = 2.0 * m * n * k
+    peak_i8 = bf16_tf * INT8_OVER_BF16
+    # the kernel's bound: HBM below the ridge point (int8 ops per byte at
+    # which the tensor peak and the HBM peak take equal time), tensor above
+    hbm_bound = is_hbm_bound(m, k, n, fmt, fused)
+    on_tc = args.path == "tc" or (args.path == "auto" and m > 8)
+    kname = ("gemv_kernel (fused act, one launch per step)" if fused else
+             "gemm_tc_kernel (tcgen05 kind::i8)" if on_tc else "gemv_kernel")
+    kfiles = ["gemm_tc.cuh", "iq8r_device.cuh"] if on_tc else ["gemv.cuh", "act_quant.cuh", "iq8r_device.cuh"]
+    ktraffic = recorded_traffic("gemm_tc_kernel" if on_tc else "gemv_kernel", args.config, kfiles)
+    if hbm_bound:
         achieved = lin_b / (lin_avg_ms * 1e-3) / 1e9
-        roof = {"bound": "hbm", "kernel": "gemv_kernel (fused act, one launch per step)", "achieved": achieved,
+        roof = {"bound": "hbm", "kernel": kname, "achieved": achieved,
                 "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "peak_source": f"{peak_src} HBM copy (MEASURED_PEAKS.json hbm_gbs)"
                 if peak_src == "measured" else "fallback 6.65 TB/s",
-                "traffic": recorded_traffic("gemv_kernel", args.config, kern_files),
-                "algorithmic_bytes_per_launch": lin_b, "avg_launch_ms": lin_avg_ms}
+                "traffic": ktraffic,
+                "algorithmic_bytes_per_launch": lin_b, "avg_launch_ms": lin_avg_ms,
+                "int8_tops": ops / (lin_avg_ms * 1e-3) / 1e12}
     else:
         # a dense int8 contraction on the tensor cores: its roofline is the int8
         # tensor peak, the measured bf16 peak times the nominal int8/bf16 ratio
-        ops = 2.0 * m * n * k
-        peak_i8 = bf16_tf * INT8_OVER_BF16
         achieved_t = ops / (lin_avg_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "kernel": "gemm_tc_kernel (tcgen05 kind::i8)", "achieved": achieved_t,
+        roof = {"bound": "tensor", "kernel": kname, "achieved": achieved_t,
                 "peak": peak_i8, "unit": "TOPS", "frac": achieved_t / peak_i8,
                 "peak_source": (f"{peak_src} cuBLAS bf16 {bf16_tf:.1f} TFLOP/s (MEASURED_PEAKS.json bf16_tflops) "
                                 f"x {INT8_OVER_BF16:g} (nominal dense int8/bf16)"),
                 "frac_of_datasheet_4500": achieved_t / 4500.0,
                 "hbm_gbs": lin_b / (lin_avg_ms * 1e-3) / 1e9,
-                "traffic": recorded_traffic("gemm_tc_kernel", args.config, ["gemm_tc.cuh", "iq8r_device.cuh"]),
+                "traffic": ktraffic,
                 "algorithmic_ops_per_launch": ops, "algorithmic_bytes_per_launch": lin_b,
                 "avg_launch_ms": lin_avg_ms}
     if not fused:
@@ -403,10 +442,10 @@ def run_ours(args, rank, world, local_rank):
                               "achieved_gbs": act_bytes(m, k) / (act_avg_ms * 1e-3) / 1e9,
                               "frac_of_hbm": act_bytes(m, k) / (act_avg_ms * 1e-3) / 1e9 / hbm}
 
-    value = world * step_bytes(m, k, n, fmt) * K / (elapsed_ms * 1e-3) / 1e9
+    value = job_value(step_bytes(m, k, n, fmt, fused) * K, world, elapsed_ms) / 1e9
     unit = "GB/s"
-    if m > 8:  # prefill-like steps are reported in int8 TOPS
-        value = world * 2.0 * m * n * k * K / (elapsed_ms * 1e-3) / 1e12
+    if not hbm_bound:  # tensor-bound (prefill) steps are reported in int8 TOPS
+        value = job_value(ops * K, world, elapsed_ms) / 1e12
         unit = "TOPS"
     clocks = sampler.summary(t_start_wall, t_end_wall)
     out = {
@@ -415,7 +454,7 @@ def run_ours(args, rank, world, local_rank):
         "dtype": "int8", "data": "synthetic",
         "config": {"workload": args.config, "m": m, "k": k, "n": n, "format": fmt, "rotated": True,
                    "step": "iq8r_linear_bf16 (one launch)" if fused else "iq8r_rotate_quant_act + iq8r_linear",
-                   "bytes_per_step": step_bytes(m, k, n, fmt),
+                   "bytes_per_step": step_bytes(m, k, n, fmt, fused), "path": args.path,
                    "l2": f"{R} rotating weight/input copies ({R * footprint / 1e6:.0f} MB > 3x L2)" if R > 1
                    else "a step moves more than 3x L2",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
@@ -447,7 +486,9 @@ def run_oracle(cfg_name, budget_s, steps=None):
 
     A sample step is the oracle's act_quant over all M tokens plus its
     linear over a slice of the N weight rows, sized to the budget. Returns
-    (value in GB/s of algorithmic bytes, sample description, steps, s/step).
+    (value, unit, sample description, steps, s/step), the value in the
+    workload's own unit: GB/s of algorithmic bytes for HBM-bound workloads,
+    int8 TOPS (2 M N K per step) for tensor-bound ones.
     """
     import oracle
     from iq8r_inputs import WORKLOADS, gen_workload
@@ -476,10 +517,14 @@ def run_oracle(cfg_name, budget_s, steps=None):
         q, a = oracle.act_quant(x)
         oracle.linear(q, a, fmt, *packed, rotated=True)
     dt = time.perf_counter() - t
-    b = step_bytes(m_s, k, n_s, fmt)
+    if is_hbm_bound(m, k, n, fmt):
+        b = step_bytes(m_s, k, n_s, fmt, fused=m <= 8)
+        value, unit, what = b * reps / dt / 1e9, "GB/s", "algorithmic bytes"
+    else:
+        value, unit, what = 2.0 * m_s * n_s * k * reps / dt / 1e12, "TOPS", "int8 ops (2 M N K)"
     sample = (f"{reps} oracle steps of act_quant over {m_s} tokens + linear over {n_s} of {n} weight rows "
-              f"(K={k}, {fmt}); value = algorithmic bytes of that slice per second")
-    return b * reps / dt / 1e9, sample, reps, dt / reps
+              f"(K={k}, {fmt}); value = {what} of that slice per second")
+    return value, unit, sample, reps, dt / reps
 
 
 def run_reference(args, rank, world):
@@ -488,15 +533,15 @@ def run_reference(args, rank, world):
     budget = float(os.environ.get("IQ8R_REF_BUDGET_S", "60"))
     # warm-up: W oracle steps of the same slice, untimed, within the budget
     run_oracle(args.config, min(budget / 10, 5.0), steps=max(1, min(W, 3)))
-    value, sample, reps, s_per = run_oracle(args.config, budget, steps=K)
+    value, unit, sample, reps, s_per = run_oracle(args.config, budget, steps=K)
     cores = blas_threads()
     return {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": K, "warmup": W,
         "ms_per_step": s_per * 1e3, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "int8", "data": "synthetic", "impl": "reference",
         "config": {"workload": args.config, "m": m, "k": k, "n": n, "format": fmt, "rotated": True},
-        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample},
-        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": value, "unit": unit, "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
@@ -509,6 +554,8 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", choices=sorted(CONFIGS), default="decode")
+    ap.add_argument("--path", choices=["auto", "gemv", "tc"], default="auto",
+                    help="force the linear's kernel (auto: the library's choice)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill TOPS line of the decode run")
@@ -549,8 +596,8 @@ def main(argv=None):
             out["prefill"] = {k_: pre[k_] for k_ in ("value", "unit", "steps", "warmup", "ms_per_step", "config",
                                                        "roofline", "gpu_launches", "clocks")}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
-            value, sample, reps, _ = run_oracle(args.config, args.cpu_budget_s)
-            out["cpu_baseline"] = {"value": value, "unit": "GB/s", "cores": blas_threads(), "kind": "oracle",
+            value, unit, sample, reps, _ = run_oracle(args.config, args.cpu_budget_s)
+            out["cpu_baseline"] = {"value": value, "unit": unit, "cores": blas_threads(), "kind": "oracle",
                                    "sample": sample}
         if rank == 0:
             print(json.dumps(out), flush=True)

@@ -126,6 +126,65 @@ __global__ void __launch_bounds__(128) act_quant_reg_kernel(const uint16_t* __re
   if (threadIdx.x == 0) xs[row] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
 }
 
+// Few tokens: a row is shared by the C CTAs of one thread-block cluster
+// (blockIdx.x = part of the row, blockIdx.y = token), each holding whole
+// 128-chunks in registers (J slots per thread). The token's amax is the max
+// of the C CTA maxima, read from each other's shared memory (DSMEM), so the
+// row is read from HBM once and C SMs share it.
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float ld_shared_cluster_f32(const float* p, uint32_t rank) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(smem_addr(p)), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(remote) : "memory");
+  return v;
+}
+
+template <int J>
+__global__ void __launch_bounds__(1024) act_quant_cluster_kernel(const uint16_t* __restrict__ x, int k,
+                                                                 int slots_per_part, int rotate,
+                                                                 int8_t* __restrict__ xq, float* __restrict__ xs) {
+  __shared__ float red[32];
+  __shared__ float part_max;
+  const int64_t row = blockIdx.y;
+  const int slots = k / kActSlot;
+  const int lane = threadIdx.x & 31;
+  const int s0 = blockIdx.x * slots_per_part;
+  const int s1 = min(slots, s0 + slots_per_part);
+  const uint16_t* xr = x + row * k;
+  float v[J][kActSlot];
+  float amax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int s = s0 + threadIdx.x + j * blockDim.x;
+    if (s < s1) {
+      act_load_slot(xr + s * kActSlot, v[j], true);
+    } else {
+#pragma unroll
+      for (int i = 0; i < kActSlot; ++i) v[j][i] = 0.0f;
+    }
+    if (rotate) act_fwht_slot(v[j], lane);  // parts and J-steps hold whole 8-lane groups
+    amax = fmaxf(amax, act_slot_absmax(v[j]));
+  }
+  amax = act_block_max(amax, red);
+  if (threadIdx.x == 0) part_max = amax;
+  cluster_sync_all();  // every part's maximum is in its shared memory
+  float g = 0.0f;
+  for (uint32_t r = 0; r < gridDim.x; ++r) g = fmaxf(g, ld_shared_cluster_f32(&part_max, r));
+  cluster_sync_all();  // no CTA leaves while another still reads its maximum
+  const float inv = g > 0.0f ? __fdiv_rn(127.0f, g) : 0.0f;
+  int8_t* qr = xq + row * k;
+#pragma unroll
+  for (int j = 0; j < J; ++j) {
+    const int s = s0 + threadIdx.x + j * blockDim.x;
+    if (s < s1) act_store_slot(qr + s * kActSlot, v[j], inv);
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) xs[row] = g > 0.0f ? __fdiv_rn(g, 127.0f) : 0.0f;
+}
+
 // Any K: pass 1 finds amax, pass 2 reloads the row (now in L2), repeats the
 // identical transform and quantises.
 __global__ void __launch_bounds__(kActTwoPassThreads) act_quant_2pass_kernel(const uint16_t* __restrict__ x, int k,

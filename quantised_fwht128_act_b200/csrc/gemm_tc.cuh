@@ -16,10 +16,11 @@
 //    (128-byte swizzle) into a 4-stage ring, activations evict-last in L2
 //    (they are reused by every weight tile); the output is stored streaming
 //    (evict-first) so it does not push out weight tiles other CTAs still read;
-//  - warp 1 owns the tensor memory: it allocates two int32 accumulators of BM
-//    columns and one lane issues tcgen05.mma (4 per stage, K = 32 each),
-//    always accumulating, alternating accumulators per block and
-//    committing to mbarriers;
+//  - warp 1 owns the tensor memory: it allocates 2..8 int32 accumulators of
+//    BM columns (as many as 512 columns hold, so the epilogue may lag several
+//    blocks behind on small tiles) and one lane issues tcgen05.mma (4 per
+//    stage, K = 32 each), always accumulating, one accumulator per 256-K block
+//    in turn, committing to mbarriers;
 //  - warps 2..9 are the epilogue: warp e covers TMEM lanes 32 (warp % 4) of
 //    column group e / 4 (half the tile's tokens). The accumulators start each block at the bits of
 //    1.5 * 2^23, so the int32 sums read back (tcgen05.ld) are the floats
@@ -39,17 +40,21 @@ namespace iq8r {
 constexpr int kTcBN = 128;            // weight rows per tile (MMA M)
 constexpr int kTcMaxBM = 256;         // tokens per tile (MMA N)
 constexpr int kTcStageK = 128;        // K bytes per stage: one 128-byte swizzle row
-constexpr int kTcStages = 4;
+constexpr int kTcStages = 4;          // stages of the largest (BM = 256) stage size
+constexpr int kTcMaxStages = 12;      // smaller token tiles get more, smaller stages
+constexpr int kTcMaxAcc = 8;          // TMEM accumulators: 512 columns / bm, at most 8
 constexpr int kTcEpiWarps = 8;                 // 4 TMEM lane quarters x kTcGroups column groups
 constexpr int kTcGroups = kTcEpiWarps / 4;
 constexpr int kTcThreads = (2 + kTcEpiWarps) * 32;
-constexpr int kTcColsPerGroup = kTcMaxBM / kTcGroups;  // tokens per epilogue column group
 constexpr int kTcStageA = kTcBN * kTcStageK;                // 16 KB
 constexpr int kTcStageB = kTcMaxBM * kTcStageK;             // 32 KB
 constexpr int kTcStageBytes = kTcStageA + kTcStageB;        // 48 KB
-// stages, then barriers (13 x 8 B), the TMEM address, 2 x 256 activation
-// scales; plus 1 KB to align the stages to 1024 bytes
-constexpr int kTcSmemBytes = kTcStages * kTcStageBytes + 4096 + 1024;
+constexpr int kTcRingBytes = kTcStages * kTcStageBytes;     // 192 KB for the operand ring
+// ring, then barriers (2 x 12 + 2 x 8 + 1) x 8 B, the TMEM address and flags, 2 x 256
+// activation scales; plus 1 KB to align the ring to 1024 bytes
+constexpr int kTcSmemBytes = kTcRingBytes + 4096 + 1024;
+// Split-K partial tiles: fp32 [BM][128] per unit, BM <= 128 when split.
+constexpr int kTcSplitMaxBM = 128;
 
 struct TcParams {
   int64_t m;          // tokens
@@ -59,7 +64,15 @@ struct TcParams {
   int fmt;            // 0 trunk, 1 lm_head
   int rotated;
   int64_t tiles_m;    // token tiles
-  int64_t tiles;      // total tiles
+  int64_t tiles;      // output tiles (tiles_m x weight tiles)
+  int splits;         // K ranges per tile (split-K), >= 1; a unit is (tile, split)
+  int64_t units;      // tiles x splits
+  int stages;         // operand ring depth (stage = 16 KB weights + bm x 128 tokens)
+  int nacc;           // TMEM accumulators of bm columns (2 .. kTcMaxAcc)
+  int stage_bytes;
+  int stream_w;       // 1: weights are read once (one token tile): evict-first
+  float* ws;          // split > 1: fp32 [units][bm][128] partial tiles
+  int* counters;      // split > 1: [tiles] arrivals, zero between calls
   const float* xs;    // [m] activation scales
   const uint8_t* sub; // [n][k/256]
   const uint16_t* scale;  // [n] or [n][k/128]
@@ -184,39 +197,46 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 
 // ------------------------------------------------------------------ kernel
 
-template <int FMT, bool PARTIALS>
+// BMAX: the largest token tile the instance handles (256, or 128 for the
+// split-K capable instance, whose epilogue keeps half the registers).
+template <int FMT, bool PARTIALS, int BMAX>
 __global__ void __launch_bounds__(kTcThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                    const TcParams p) {
+  constexpr int kCols = BMAX / kTcGroups;  // most tokens per epilogue column group
+  constexpr bool kCanSplit = BMAX <= kTcSplitMaxBM && !PARTIALS;
   constexpr int G = FMT == 0 ? kGroupTrunk : kGroupHead;
   constexpr int SPB = G / kTcStageK;  // stages per scale block: 2 (trunk) or 1 (lm_head)
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment for the swizzled TMA tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTcStages * kTcStageBytes);
-  uint64_t* empty = full + kTcStages;
-  uint64_t* acc_full = empty + kTcStages;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* mma_done = acc_empty + 2;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTcRingBytes);
+  uint64_t* empty = full + kTcMaxStages;
+  uint64_t* acc_full = empty + kTcMaxStages;
+  uint64_t* acc_empty = acc_full + kTcMaxAcc;
+  uint64_t* mma_done = acc_empty + kTcMaxAcc;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
+  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sa = reinterpret_cast<float*>(tmem_slot + 4);  // [2][kTcMaxBM] activation scales per tile
   __shared__ volatile int s_abort;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int K = p.k;
-  const int nkb = K / kTcStageK;       // stages per tile
   const int ng = K / G;                // scale blocks per row
   const int bm = p.bm;
+  const int S = kCanSplit ? p.splits : 1;  // instances that never split keep the plain tile loop
+  const int nst = p.stages;
+  const int nacc = p.nacc;
 
   if (threadIdx.x == 0) {
     s_abort = 0;
-    for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
+    for (int st = 0; st < nst; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < nacc; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kTcEpiWarps);
     }
@@ -234,76 +254,102 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  // A unit is one output tile over one K range: blocks [g0, g1) of the tile's
+  // ng scale blocks, split s of S (the tile's K split evenly in blocks).
+  auto unit_range = [&](int64_t u, int64_t& tile, int& split, int& g0, int& g1) {
+    tile = u / S;
+    split = static_cast<int>(u - tile * S);
+    g0 = static_cast<int>((static_cast<int64_t>(split) * ng) / S);
+    g1 = static_cast<int>((static_cast<int64_t>(split + 1) * ng) / S);
+  };
+
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint64_t pol_w = l2_policy_evict_normal();
+      const uint64_t pol_w = p.stream_w ? l2_policy_evict_first() : l2_policy_evict_normal();
       const uint64_t pol_x = l2_policy_evict_last();
       const uint32_t tx = kTcStageA + bm * kTcStageK;
-      uint32_t it = 0;
+      uint32_t it = 0;   // stages issued
+      int st = 0;        // ring slot of stage `it`
+      uint32_t ph = 0;   // its use count & 1
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
+      for (int64_t u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        int64_t tile;
+        int split, g0, g1;
+        unit_range(u, tile, split, g0, g1);
         const int m0 = static_cast<int>((tile % p.tiles_m) * bm);
         const int n0 = static_cast<int>((tile / p.tiles_m) * kTcBN);
-        for (int kb = 0; kb < nkb; ++kb, ++it) {
-          const int s = static_cast<int>(it % kTcStages);
-          const uint32_t use = it / kTcStages;
-          if (s_abort || (use > 0 && !mbar_wait(&empty[s], (use - 1) & 1u, kDevErrTcEmpty))) {
+        for (int kb = g0 * SPB; kb < g1 * SPB; ++kb, ++it) {
+          if (s_abort || (it >= static_cast<uint32_t>(nst) && !mbar_wait(&empty[st], ph ^ 1u, kDevErrTcEmpty))) {
             s_abort = 1;
             ok = false;
             break;
           }
-          uint8_t* st = stage_base + s * kTcStageBytes;
-          mbar_arrive_expect_tx(&full[s], tx);
-          tma_load_2d(st, &tmap_w, kb * kTcStageK, n0, &full[s], pol_w);
-          tma_load_2d(st + kTcStageA, &tmap_x, kb * kTcStageK, m0, &full[s], pol_x);
+          uint8_t* sp = stage_base + st * p.stage_bytes;
+          mbar_arrive_expect_tx(&full[st], tx);
+          tma_load_2d(sp, &tmap_w, kb * kTcStageK, n0, &full[st], pol_w);
+          tma_load_2d(sp + kTcStageA, &tmap_x, kb * kTcStageK, m0, &full[st], pol_x);
+          if (++st == nst) {
+            st = 0;
+            ph ^= 1u;
+          }
         }
       }
       // never leave with a copy still landing in this CTA's shared memory
-      const uint32_t first = it > static_cast<uint32_t>(kTcStages) ? it - kTcStages : 0u;
+      const uint32_t first = it > static_cast<uint32_t>(nst) ? it - nst : 0u;
       for (uint32_t j = first; j < it; ++j)
-        if (!mbar_wait(&full[j % kTcStages], (j / kTcStages) & 1u, kDevErrTcDrain)) break;
+        if (!mbar_wait(&full[j % nst], (j / nst) & 1u, kDevErrTcDrain)) break;
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       const uint32_t idesc = umma_idesc_i8(bm);
       uint32_t it = 0;   // stages consumed
-      uint32_t blk = 0;  // accumulator blocks produced
+      int st = 0;        // ring slot of stage `it`
+      uint32_t ph = 0;   // its use count & 1
+      int buf = 0;       // accumulator of the current block
+      uint32_t aph = 0;  // its use count & 1
       bool ok = true;
-      for (int64_t tile = blockIdx.x; tile < p.tiles && ok; tile += gridDim.x) {
-        for (int kb = 0; kb < nkb && ok; ++kb, ++it) {
-          const int buf = static_cast<int>(blk & 1u);
+      for (int64_t u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
+        int64_t tile;
+        int split, g0, g1;
+        unit_range(u, tile, split, g0, g1);
+        for (int kb = g0 * SPB; kb < g1 * SPB && ok; ++kb, ++it) {
           const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * bm);
           if (kb % SPB == 0) {
-            // this accumulator must have been drained by the epilogue
-            // drained by the epilogue and reset to the bias (seeded once at start)
-            const uint32_t use = blk >> 1;
-            if (s_abort || !mbar_wait(&acc_empty[buf], use & 1u, kDevErrTcAccEmpty)) {
+            // the accumulator must have been drained by the epilogue and
+            // reset to the bias (the epilogue seeds all of them at the start)
+            if (s_abort || !mbar_wait(&acc_empty[buf], aph, kDevErrTcAccEmpty)) {
               s_abort = 1;
               ok = false;
               break;
             }
             tc_fence_after();
           }
-          const int s = static_cast<int>(it % kTcStages);
-          if (s_abort || !mbar_wait(&full[s], (it / kTcStages) & 1u, kDevErrTcFull)) {
+          if (s_abort || !mbar_wait(&full[st], ph, kDevErrTcFull)) {
             s_abort = 1;
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t a_addr = smem_addr(stage_base + s * kTcStageBytes);
+          const uint32_t a_addr = smem_addr(stage_base + st * p.stage_bytes);
           const uint32_t b_addr = a_addr + kTcStageA;
 #pragma unroll
           for (int k = 0; k < kTcStageK / 32; ++k) {
             // advancing K by 32 bytes inside the swizzle atom moves the start address
             umma_i8(d_tmem, umma_desc_sw128(a_addr + 32 * k), umma_desc_sw128(b_addr + 32 * k), idesc, 1u);
           }
-          umma_commit(&empty[s]);  // the stage can be refilled once these MMAs have read it
+          umma_commit(&empty[st]);  // the stage can be refilled once these MMAs have read it
+          if (++st == nst) {
+            st = 0;
+            ph ^= 1u;
+          }
           if (kb % SPB == SPB - 1) {
             umma_commit(&acc_full[buf]);  // the block's int32 sums are complete
-            ++blk;
+            if (++buf == nacc) {
+              buf = 0;
+              aph ^= 1u;
+            }
           }
         }
       }
@@ -320,28 +366,31 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int q = e >> 2;            // column group: tokens [q * cols, (q + 1) * cols) of the tile
     const int lq = warp & 3;         // TMEM lane quarter this warp may access
     const int cols = bm / kTcGroups; // tokens per column group (a multiple of 16 when bm is of 32)
+    const int rloc = lq * 32 + lane; // this thread's row within the weight tile
     const uint32_t lane_addr = static_cast<uint32_t>(lq * 32) << 16;
     const float rot = p.rotated ? 0.0078125f : 1.0f;
-    // seed both accumulators with the bias (this warp's lanes and columns)
-    for (int b = 0; b < 2; ++b) {
+    // seed every accumulator with the bias (this warp's lanes and columns)
+    for (int b = 0; b < nacc; ++b) {
       const uint32_t t0 = tmem_base + lane_addr + static_cast<uint32_t>(b * bm + q * cols);
       for (int c = 0; c < cols; c += 16) tmem_st16_fill(t0 + c, kTcBiasBits);
     }
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) {
-      mbar_arrive(&acc_empty[0]);
-      mbar_arrive(&acc_empty[1]);
-    }
+    if (lane == 0)
+      for (int b = 0; b < nacc; ++b) mbar_arrive(&acc_empty[b]);
     const uint64_t neg_bias = f2_splat(-kTcBias);
-    uint32_t blk = 0;
+    int buf = 0;       // accumulator of the current block
+    uint32_t aph = 0;  // its use count & 1
     int par = 0;
     bool failed = false;
-    for (int64_t tile = blockIdx.x; tile < p.tiles; tile += gridDim.x, par ^= 1) {
+    for (int64_t u = blockIdx.x; u < p.units; u += gridDim.x, par ^= 1) {
+      int64_t tile;
+      int split, g0, g1;
+      unit_range(u, tile, split, g0, g1);
       const int64_t m0 = (tile % p.tiles_m) * bm;
       const int64_t n0 = (tile / p.tiles_m) * kTcBN;
-      const int64_t n = n0 + lq * 32 + lane;  // this thread's weight row
+      const int64_t n = n0 + rloc;  // this thread's weight row
       const bool nvalid = n < p.n;
       // activation scales of the tile's tokens, shared by all epilogue warps
       if (!PARTIALS) {
@@ -350,22 +399,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       float s2f = 0.0f;
       if (FMT == 0 && !PARTIALS && nvalid) s2f = bf16_bits_to_float(p.scale[n]);
-      uint64_t acc[kTcColsPerGroup / 2];  // fp32 pairs
+      uint64_t acc[kCols / 2];  // fp32 pairs
 #pragma unroll
-      for (int j = 0; j < kTcColsPerGroup / 2; ++j) acc[j] = 0ull;
+      for (int j = 0; j < kCols / 2; ++j) acc[j] = 0ull;
       // the first block's scale, then one block ahead
       float snext = 0.0f;
       if (!PARTIALS && nvalid)
-        snext = FMT == 0 ? static_cast<float>(__ldg(p.sub + n * ng)) : bf16_bits_to_float(__ldg(p.scale + n * ng));
-      for (int g = 0; g < ng; ++g, ++blk) {
+        snext = FMT == 0 ? static_cast<float>(__ldg(p.sub + n * ng + g0))
+                         : bf16_bits_to_float(__ldg(p.scale + n * ng + g0));
+      for (int g = g0; g < g1; ++g) {
         const uint64_t sg = f2_splat(snext);
-        if (!PARTIALS && nvalid && g + 1 < ng)
+        if (!PARTIALS && nvalid && g + 1 < g1)
           snext = FMT == 0 ? static_cast<float>(__ldg(p.sub + n * ng + g + 1))
                            : bf16_bits_to_float(__ldg(p.scale + n * ng + g + 1));
-        const int buf = static_cast<int>(blk & 1u);
         if (!failed) {
           bool bad = s_abort != 0;
-          if (!bad) bad = !mbar_wait(&acc_full[buf], (blk >> 1) & 1u, kDevErrTcAccFull);
+          if (!bad) bad = !mbar_wait(&acc_full[buf], aph, kDevErrTcAccFull);
           failed = !__all_sync(0xffffffffu, !bad);
           if (failed && lane == 0) s_abort = 1;
         }
@@ -373,14 +422,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t tbase = tmem_base + lane_addr + static_cast<uint32_t>(buf * bm + q * cols);
         // with few columns per thread, chunk c + 1 loads while chunk c is
         // converted and summed; with many, registers are kept for the sums
-        constexpr bool kPipe = kTcColsPerGroup <= 64;
+        constexpr bool kPipe = kCols <= 64;
         uint32_t rn[16];
         if (kPipe && !failed) {
           tmem_ld16(tbase, rn);
           tmem_wait_ld();
         }
 #pragma unroll
-        for (int c = 0; c < kTcColsPerGroup; c += 16) {
+        for (int c = 0; c < kCols; c += 16) {
           if (c < cols) {
             uint32_t r[16];
             if (kPipe) {
@@ -414,14 +463,60 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&acc_empty[buf]);
+        if (++buf == nacc) {
+          buf = 0;
+          aph ^= 1u;
+        }
       }
       if (PARTIALS) continue;
-      // all epilogue warps have staged their part of sa before anyone reads it
-      named_barrier(1, kTcEpiWarps * 32);
+      if (kCanSplit && S > 1) {
+        // split-K: publish this unit's fp32 partial tile; the tile's last
+        // unit to arrive adds all S partials in split order (the same order
+        // whichever unit is last) and writes the output
+        float* wsu = p.ws + static_cast<size_t>(u) * bm * kTcBN;
+#pragma unroll
+        for (int j = 0; j < kCols; j += 2) {
+          if (j < cols) {
+            float a0, a1;
+            f2_unpack(acc[j / 2], a0, a1);
+            __stcg(wsu + (q * cols + j) * kTcBN + rloc, a0);
+            __stcg(wsu + (q * cols + j + 1) * kTcBN + rloc, a1);
+          }
+        }
+        __threadfence();
+        named_barrier(1, kTcEpiWarps * 32);
+        if (e == 0 && lane == 0) {
+          const int prev = atomicAdd(p.counters + tile, 1);
+          const int last = prev == S - 1;
+          if (last) p.counters[tile] = 0;  // ready for the next call
+          *s_last = last;
+        }
+        named_barrier(1, kTcEpiWarps * 32);
+        if (!*s_last) continue;
+        __threadfence();
+        const float* wst = p.ws + static_cast<size_t>(tile) * S * bm * kTcBN;
+#pragma unroll
+        for (int j = 0; j < kCols; j += 2) {
+          if (j < cols) {
+            float own0, own1;
+            f2_unpack(acc[j / 2], own0, own1);
+            float t0 = 0.0f, t1 = 0.0f;
+            for (int sp = 0; sp < S; ++sp) {
+              const float* w = wst + static_cast<size_t>(sp) * bm * kTcBN + (q * cols + j) * kTcBN + rloc;
+              t0 += sp == split ? own0 : __ldcg(w);
+              t1 += sp == split ? own1 : __ldcg(w + kTcBN);
+            }
+            acc[j / 2] = u2_pack(__float_as_uint(t0), __float_as_uint(t1));
+          }
+        }
+      } else {
+        // all epilogue warps have staged their part of sa before anyone reads it
+        named_barrier(1, kTcEpiWarps * 32);
+      }
       if (!failed && nvalid) {
         const float rs = (FMT == 0 ? s2f : 1.0f) * rot;
 #pragma unroll
-        for (int j = 0; j < kTcColsPerGroup; j += 2) {
+        for (int j = 0; j < kCols; j += 2) {
           float a0, a1;
           f2_unpack(acc[j / 2], a0, a1);
           const int64_t m = m0 + q * cols + j;

@@ -3,6 +3,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <mutex>
 #include <string>
 
 #include <cudaTypedefs.h>
@@ -150,11 +151,50 @@ int gemv_max_mt(int64_t k, const DeviceInfo& d) {
 
 }  // namespace
 
+template <int J>
+cudaError_t launch_act_cluster_t(const uint16_t* x, int64_t m, int k, int parts, int slots_per_part, int threads,
+                                 int rotate, int8_t* xq, float* xs, cudaStream_t stream) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(parts), static_cast<unsigned>(m));
+  cfg.blockDim = dim3(static_cast<unsigned>(threads));
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(parts);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, act_quant_cluster_kernel<J>, x, k, slots_per_part, rotate, xq, xs);
+}
+
 cudaError_t launch_act_quant(const uint16_t* x, int64_t m, int64_t k, int rotate, int8_t* xq, float* xs,
                              cudaStream_t stream) {
   if (m == 0) return cudaSuccess;
   const int slots = static_cast<int>(k / kActSlot);
   const unsigned grid = static_cast<unsigned>(m);
+  DeviceInfo d;
+  cudaError_t e = device_info(&d);
+  if (e != cudaSuccess) return e;
+  // fewer tokens than SMs: spread each row over a cluster of up to 8 CTAs
+  const int64_t chunks = k / kRot;
+  const int parts = static_cast<int>(std::min<int64_t>({8, chunks, (d.num_sms + m - 1) / m}));
+  if (parts > 1 && m <= 65535) {
+    const int spp = static_cast<int>((chunks + parts - 1) / parts) * (kRot / kActSlot);
+    const int threads = std::min(1024, (spp + 31) / 32 * 32);
+    const int j = (spp + threads - 1) / threads;
+    const int kk = static_cast<int>(k);
+    // every part must own at least one chunk: parts * spp covers the row
+    // and (parts - 1) * spp < slots
+    if (j <= 3 && static_cast<int64_t>(parts - 1) * spp < slots) {
+      switch (j) {
+        case 1: e = launch_act_cluster_t<1>(x, m, kk, parts, spp, threads, rotate, xq, xs, stream); break;
+        case 2: e = launch_act_cluster_t<2>(x, m, kk, parts, spp, threads, rotate, xq, xs, stream); break;
+        default: e = launch_act_cluster_t<3>(x, m, kk, parts, spp, threads, rotate, xq, xs, stream); break;
+      }
+      return e;
+    }
+  }
   if (k <= kActRegMaxK) {
     const int threads = slots <= 128 ? ((slots + 31) / 32) * 32 : 128;
     const int j = (slots + threads - 1) / threads;
@@ -260,10 +300,67 @@ cudaError_t make_tmap_i8(CUtensorMap* map, const void* base, int64_t rows, int64
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <int FMT, bool PARTIALS>
+// Split-K workspace, one per device, made on the first split launch there:
+// fp32 partial tiles and per-tile arrival counters (zeroed once; the last
+// unit of every tile resets its counter).
+constexpr size_t kTcWsBytes = size_t(32) << 20;
+constexpr int64_t kTcMaxCounters = 8192;
+struct TcWorkspace {
+  float* ws = nullptr;
+  int* counters = nullptr;
+};
+TcWorkspace g_tc_ws[kMaxDevices];
+std::mutex g_tc_ws_mu;
+
+cudaError_t tc_workspace(TcWorkspace* out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_tc_ws_mu);
+  TcWorkspace& w = g_tc_ws[dev];
+  if (w.ws == nullptr) {
+    void* a = nullptr;
+    void* c = nullptr;
+    e = cudaMalloc(&a, kTcWsBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaMalloc(&c, kTcMaxCounters * sizeof(int));
+    if (e == cudaSuccess) e = cudaMemset(c, 0, kTcMaxCounters * sizeof(int));
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) {
+      cudaFree(a);
+      if (c) cudaFree(c);
+      return e;
+    }
+    w.ws = static_cast<float*>(a);
+    w.counters = static_cast<int*>(c);
+  }
+  *out = w;
+  return cudaSuccess;
+}
+
+// Cost, in scale blocks, of the busiest CTA when `units` units of a tile
+// split S ways are dealt round-robin to min(sms, units) persistent CTAs;
+// a split unit also pays about one block for its partial tile.
+double tc_split_cost(int64_t tiles, int ng, int S, int sms) {
+  const int64_t units = tiles * S;
+  const int64_t grid = std::min<int64_t>(sms, units);
+  double worst = 0.0;
+  for (int64_t c = 0; c < grid; ++c) {
+    double t = 0.0;
+    for (int64_t u = c; u < units; u += grid) {
+      const int64_t sp = u % S;
+      t += static_cast<double>((sp + 1) * ng / S - sp * ng / S) + 0.25 + (S > 1 ? 1.0 : 0.0);
+    }
+    worst = std::max(worst, t);
+  }
+  return worst;
+}
+
+template <int FMT, bool PARTIALS, int BMAX>
 cudaError_t launch_tc_t(const CUtensorMap& tw, const CUtensorMap& tx, const TcParams& p, int grid,
                         cudaStream_t stream) {
-  auto kernel = gemm_tc_kernel<FMT, PARTIALS>;
+  auto kernel = gemm_tc_kernel<FMT, PARTIALS, BMAX>;
   static std::atomic<int> configured[kMaxDevices];
   cudaError_t e = ensure_smem(kernel, kTcSmemBytes, configured);
   if (e != cudaSuccess) return e;
@@ -306,23 +403,59 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream) {
   p.rotated = a.rotated;
   p.tiles_m = (a.m + p.bm - 1) / p.bm;
   p.tiles = p.tiles_m * ((a.n + kTcBN - 1) / kTcBN);
+  p.stage_bytes = kTcStageA + p.bm * kTcStageK;
+  p.stages = std::min(kTcMaxStages, kTcRingBytes / p.stage_bytes);
+  p.stream_w = p.tiles_m == 1 ? 1 : 0;
+  // split K when there are too few tiles to fill the SMs
+  const int ng = static_cast<int>(a.k / (a.fmt == 0 ? kGroupTrunk : kGroupHead));
+  p.splits = 1;
+  if (p.bm <= kTcSplitMaxBM && p.tiles <= kTcMaxCounters && a.partials == nullptr) {
+    double best = tc_split_cost(p.tiles, ng, 1, d.num_sms);
+    for (int S = 2; S <= std::min(ng, 32); ++S) {
+      if (static_cast<size_t>(p.tiles) * S * p.bm * kTcBN * sizeof(float) > kTcWsBytes) break;
+      const double c = tc_split_cost(p.tiles, ng, S, d.num_sms);
+      if (c < 0.95 * best) {
+        best = c;
+        p.splits = S;
+      }
+    }
+  }
+  p.units = p.tiles * p.splits;
+  if (p.splits > 1) {
+    TcWorkspace w;
+    e = tc_workspace(&w);
+    if (e != cudaSuccess) return e;
+    p.ws = w.ws;
+    p.counters = w.counters;
+  }
   p.xs = a.xs;
   p.sub = a.sub;
   p.scale = a.scale;
   p.y = a.y;
   p.partials = a.partials;
+  p.nacc = std::max(2, std::min(kTcMaxAcc, 512 / p.bm));
   uint32_t cols = 32;
-  while (cols < static_cast<uint32_t>(2 * p.bm)) cols <<= 1;
+  while (cols < static_cast<uint32_t>(p.nacc * p.bm)) cols <<= 1;
   p.tmem_cols = cols;
   CUtensorMap tw, tx;
   e = make_tmap_i8(&tw, a.codes, a.n, a.k, kTcBN);
   if (e != cudaSuccess) return e;
   e = make_tmap_i8(&tx, a.xq, a.m, a.k, p.bm);
   if (e != cudaSuccess) return e;
-  const int grid = static_cast<int>(std::min<int64_t>(d.num_sms, p.tiles));
+  const int grid = static_cast<int>(std::min<int64_t>(d.num_sms, p.units));
   const bool part = a.partials != nullptr;
-  if (a.fmt == 0) return part ? launch_tc_t<0, true>(tw, tx, p, grid, stream) : launch_tc_t<0, false>(tw, tx, p, grid, stream);
-  return part ? launch_tc_t<1, true>(tw, tx, p, grid, stream) : launch_tc_t<1, false>(tw, tx, p, grid, stream);
+  if (p.bm <= kTcSplitMaxBM) {
+    if (a.fmt == 0)
+      return part ? launch_tc_t<0, true, kTcSplitMaxBM>(tw, tx, p, grid, stream)
+                  : launch_tc_t<0, false, kTcSplitMaxBM>(tw, tx, p, grid, stream);
+    return part ? launch_tc_t<1, true, kTcSplitMaxBM>(tw, tx, p, grid, stream)
+                : launch_tc_t<1, false, kTcSplitMaxBM>(tw, tx, p, grid, stream);
+  }
+  if (a.fmt == 0)
+    return part ? launch_tc_t<0, true, kTcMaxBM>(tw, tx, p, grid, stream)
+                : launch_tc_t<0, false, kTcMaxBM>(tw, tx, p, grid, stream);
+  return part ? launch_tc_t<1, true, kTcMaxBM>(tw, tx, p, grid, stream)
+              : launch_tc_t<1, false, kTcMaxBM>(tw, tx, p, grid, stream);
 }
 
 namespace {

@@ -71,7 +71,10 @@ def test_act_bit_exact_prefill_full():
     assert_act_exact(x)
 
 
-@pytest.mark.parametrize("m,k", [(5, 128), (3, 640), (7, 2176), (1, 16384), (2, 16512), (3, 33024), (33, 1152)])
+# small M: a row spread over a cluster of CTAs; M >= 148: one CTA a row, the
+# row in registers up to K = 16384, two passes above
+@pytest.mark.parametrize("m,k", [(5, 128), (3, 640), (7, 2176), (1, 16384), (2, 16512), (3, 33024), (33, 1152),
+                                 (16, 17408), (147, 256), (148, 5120), (160, 16512)])
 def test_act_bit_exact_ragged_shapes(m, k):
     x, _ = gen_workload("decode", m=m, n=8, k=k, seed=m * 1000 + k)
     assert_act_exact(x)
@@ -345,6 +348,35 @@ def test_tc_lm_head_format():
     assert np.array_equal(gpu_partials(x, W, path=iq8r.IQ8R_PATH_TC), oracle.partials(xq, codes, 128))
     y64 = oracle_linear(x, fmt, packed)
     check_output(gpu_linear(x, W, path=iq8r.IQ8R_PATH_TC), y64, oracle.linear_bf16(y64))
+
+
+# few output tiles and long K: the tile's K range is split over several CTAs
+# and the fp32 partial tiles are added by the tile's last unit
+TC_SPLIT_SHAPES = [(16, 256, 17408), (128, 384, 8192), (8, 200, 4096), (40, 130, 2560), (96, 1, 1024)]
+
+
+@pytest.mark.parametrize("m,n,k", TC_SPLIT_SHAPES)
+def test_tc_split_k_linear_within_tolerance(m, n, k):
+    x, _, fmt, packed, W = case("decode", m=m, n=n, k=k, seed=81 + m + n + k)
+    y64 = oracle_linear(x, fmt, packed)
+    y = gpu_linear(x, W, path=iq8r.IQ8R_PATH_TC)
+    st = check_output(y, y64, oracle.linear_bf16(y64))
+    assert st["bit_equal_frac"] > 0.98
+
+
+def test_tc_split_k_repeatable_and_lm_head():
+    """Back-to-back split calls give identical bits (the arrival counters
+    return to zero, the reduction order is fixed); the lm_head format splits
+    the same way."""
+    x, _, fmt, packed, W = case("decode", m=16, n=256, k=17408, seed=82)
+    xq, xs = iq8r.iq8r_rotate_quant_act(dev_bf16(x))
+    ys = [iq8r.iq8r_linear_ex(xq, xs, W, path=iq8r.IQ8R_PATH_TC) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert all(torch.equal(ys[0], y) for y in ys[1:])
+    x, _, fmt, packed, W = case("lm_head8", m=8, n=256, k=5120, seed=83)
+    y64 = oracle_linear(x, fmt, packed)
+    check_output(gpu_linear(x, W, path=iq8r.IQ8R_PATH_TC), y64, oracle.linear_bf16(y64))
+    iq8r.iq8r_get_device_error()  # raises if a kernel reported a timeout
 
 
 def test_tc_and_gemv_agree_on_partials():
