@@ -97,6 +97,7 @@ template <int J>
 __global__ void __launch_bounds__(128) act_quant_reg_kernel(const uint16_t* __restrict__ x, int k, int rotate,
                                                             int8_t* __restrict__ xq, float* __restrict__ xs) {
   __shared__ float red[32];
+  pdl_launch_dependents();  // the next kernel may start its set-up
   const int64_t row = blockIdx.x;
   const int slots = k / kActSlot;
   const int lane = threadIdx.x & 31;
@@ -148,6 +149,7 @@ __global__ void __launch_bounds__(1024) act_quant_cluster_kernel(const uint16_t*
                                                                  int slots_per_part, int rotate,
                                                                  int8_t* __restrict__ xq, float* __restrict__ xs) {
   __shared__ float red[32];
+  pdl_launch_dependents();  // the next kernel may start its set-up
   __shared__ float part_max;
   const int64_t row = blockIdx.y;
   const int slots = k / kActSlot;
@@ -191,6 +193,7 @@ __global__ void __launch_bounds__(kActTwoPassThreads) act_quant_2pass_kernel(con
                                                                              int rotate, int8_t* __restrict__ xq,
                                                                              float* __restrict__ xs) {
   __shared__ float red[32];
+  pdl_launch_dependents();  // the next kernel may start its set-up
   const int64_t row = blockIdx.x;
   const int slots = k / kActSlot;
   const int lane = threadIdx.x & 31;

@@ -71,8 +71,7 @@ struct TcParams {
   int nacc;           // TMEM accumulators of bm columns (2 .. kTcMaxAcc)
   int stage_bytes;
   int stream_w;       // 1: weights are read once (one token tile): evict-first
-  float* ws;          // split > 1: fp32 [units][bm][128] partial tiles
-  int* counters;      // split > 1: [tiles] arrivals, zero between calls
+  float* ws;          // split > 1: fp32 [units][128][bm] partial tiles
   const float* xs;    // [m] activation scales
   const uint8_t* sub; // [n][k/256]
   const uint16_t* scale;  // [n] or [n][k/128]
@@ -217,7 +216,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint64_t* acc_empty = acc_full + kTcMaxAcc;
   uint64_t* mma_done = acc_empty + kTcMaxAcc;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mma_done + 1);
-  volatile int* s_last = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* sa = reinterpret_cast<float*>(tmem_slot + 4);  // [2][kTcMaxBM] activation scales per tile
   __shared__ volatile int s_abort;
 
@@ -253,6 +251,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // set-up above overlaps the previous kernel's tail; its outputs (the
+  // activation codes and scales) are read only after it has completed
+  pdl_launch_dependents();
+  pdl_wait();
 
   // A unit is one output tile over one K range: blocks [g0, g1) of the tile's
   // ng scale blocks, split s of S (the tile's K split evenly in blocks).
@@ -369,6 +371,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const int rloc = lq * 32 + lane; // this thread's row within the weight tile
     const uint32_t lane_addr = static_cast<uint32_t>(lq * 32) << 16;
     const float rot = p.rotated ? 0.0078125f : 1.0f;
+    constexpr int kSD = BMAX >= 256 ? 4 : 8;  // blocks of scale prefetch
+    auto load_scale = [&](int64_t i) -> uint32_t {
+      return FMT == 0 ? static_cast<uint32_t>(__ldg(p.sub + i)) : static_cast<uint32_t>(__ldg(p.scale + i));
+    };
     // seed every accumulator with the bias (this warp's lanes and columns)
     for (int b = 0; b < nacc; ++b) {
       const uint32_t t0 = tmem_base + lane_addr + static_cast<uint32_t>(b * bm + q * cols);
@@ -402,16 +408,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       uint64_t acc[kCols / 2];  // fp32 pairs
 #pragma unroll
       for (int j = 0; j < kCols / 2; ++j) acc[j] = 0ull;
-      // the first block's scale, then one block ahead
-      float snext = 0.0f;
-      if (!PARTIALS && nvalid)
-        snext = FMT == 0 ? static_cast<float>(__ldg(p.sub + n * ng + g0))
-                         : bf16_bits_to_float(__ldg(p.scale + n * ng + g0));
-      for (int g = g0; g < g1; ++g) {
-        const uint64_t sg = f2_splat(snext);
-        if (!PARTIALS && nvalid && g + 1 < g1)
-          snext = FMT == 0 ? static_cast<float>(__ldg(p.sub + n * ng + g + 1))
-                           : bf16_bits_to_float(__ldg(p.scale + n * ng + g + 1));
+      // the row's block scales, loaded kSD blocks ahead of use: while the
+      // weight stream keeps HBM busy a scattered load takes microseconds
+      uint32_t sq[kSD];
+#pragma unroll
+      for (int i = 0; i < kSD; ++i) sq[i] = (!PARTIALS && nvalid && g0 + i < g1) ? load_scale(n * ng + g0 + i) : 0u;
+      for (int gb = g0; gb < g1; gb += kSD)
+#pragma unroll
+      for (int i = 0; i < kSD; ++i) {
+        const int g = gb + i;
+        if (g >= g1) break;
+        const uint64_t sg = f2_splat(FMT == 0 ? static_cast<float>(sq[i]) : bf16_bits_to_float(static_cast<uint16_t>(sq[i])));
+        if (!PARTIALS && nvalid && g + kSD < g1) sq[i] = load_scale(n * ng + g + kSD);
         if (!failed) {
           bool bad = s_abort != 0;
           if (!bad) bad = !mbar_wait(&acc_full[buf], aph, kDevErrTcAccFull);
@@ -470,49 +478,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       }
       if (PARTIALS) continue;
       if (kCanSplit && S > 1) {
-        // split-K: publish this unit's fp32 partial tile; the tile's last
-        // unit to arrive adds all S partials in split order (the same order
-        // whichever unit is last) and writes the output
-        float* wsu = p.ws + static_cast<size_t>(u) * bm * kTcBN;
+        // split-K: publish this unit's fp32 partial tile, row-major [128][bm]
+        // (this thread's row, its column group: cols consecutive floats); a
+        // second kernel adds the S partials of every tile in split order
+        float* wsu = p.ws + static_cast<size_t>(u) * kTcBN * bm + static_cast<size_t>(rloc) * bm + q * cols;
 #pragma unroll
-        for (int j = 0; j < kCols; j += 2) {
+        for (int j = 0; j < kCols; j += 4) {
           if (j < cols) {
-            float a0, a1;
+            float a0, a1, a2, a3;
             f2_unpack(acc[j / 2], a0, a1);
-            __stcg(wsu + (q * cols + j) * kTcBN + rloc, a0);
-            __stcg(wsu + (q * cols + j + 1) * kTcBN + rloc, a1);
+            f2_unpack(acc[j / 2 + 1], a2, a3);
+            __stcg(reinterpret_cast<float4*>(wsu + j), make_float4(a0, a1, a2, a3));
           }
         }
-        __threadfence();
-        named_barrier(1, kTcEpiWarps * 32);
-        if (e == 0 && lane == 0) {
-          const int prev = atomicAdd(p.counters + tile, 1);
-          const int last = prev == S - 1;
-          if (last) p.counters[tile] = 0;  // ready for the next call
-          *s_last = last;
-        }
-        named_barrier(1, kTcEpiWarps * 32);
-        if (!*s_last) continue;
-        __threadfence();
-        const float* wst = p.ws + static_cast<size_t>(tile) * S * bm * kTcBN;
-#pragma unroll
-        for (int j = 0; j < kCols; j += 2) {
-          if (j < cols) {
-            float own0, own1;
-            f2_unpack(acc[j / 2], own0, own1);
-            float t0 = 0.0f, t1 = 0.0f;
-            for (int sp = 0; sp < S; ++sp) {
-              const float* w = wst + static_cast<size_t>(sp) * bm * kTcBN + (q * cols + j) * kTcBN + rloc;
-              t0 += sp == split ? own0 : __ldcg(w);
-              t1 += sp == split ? own1 : __ldcg(w + kTcBN);
-            }
-            acc[j / 2] = u2_pack(__float_as_uint(t0), __float_as_uint(t1));
-          }
-        }
-      } else {
-        // all epilogue warps have staged their part of sa before anyone reads it
-        named_barrier(1, kTcEpiWarps * 32);
+        continue;
       }
+      // all epilogue warps have staged their part of sa before anyone reads it
+      named_barrier(1, kTcEpiWarps * 32);
       if (!failed && nvalid) {
         const float rs = (FMT == 0 ? s2f : 1.0f) * rot;
 #pragma unroll
@@ -534,6 +516,59 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(p.tmem_cols)
                  : "memory");
+  }
+}
+
+// Split-K second pass: y[m][n] = bf16(sum over splits, in split order, of
+// the fp32 partial tiles, times a[m] * s2[n] / 128 (trunk) or a[m] / 128
+// (lm_head)). One thread: one weight row of one tile, 8 consecutive tokens;
+// consecutive threads take consecutive rows, so output stores coalesce.
+constexpr int kTcReduceThreads = 256;
+template <int FMT>
+__global__ void __launch_bounds__(kTcReduceThreads) tc_split_reduce_kernel(const TcParams p) {
+  pdl_wait();  // the partial tiles come from the kernel before
+  const int chunks = p.bm / 8;
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= p.tiles * kTcBN * chunks) return;
+  const int64_t tile = i / (kTcBN * chunks);
+  const int rem = static_cast<int>(i - tile * kTcBN * chunks);
+  const int r = rem % kTcBN;
+  const int ch = rem / kTcBN;
+  const int64_t m0 = (tile % p.tiles_m) * p.bm + ch * 8;
+  const int64_t n = (tile / p.tiles_m) * kTcBN + r;
+  if (n >= p.n || m0 >= p.m) return;
+  const size_t sstride = static_cast<size_t>(kTcBN) * p.bm;
+  const float* w = p.ws + static_cast<size_t>(tile) * p.splits * sstride + static_cast<size_t>(r) * p.bm + ch * 8;
+  float acc[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+  for (int sp0 = 0; sp0 < p.splits; sp0 += 4) {
+    float4 v[4][2];
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      if (sp0 + t < p.splits) {
+        const float4* q = reinterpret_cast<const float4*>(w + (sp0 + t) * sstride);
+        v[t][0] = __ldcg(q);
+        v[t][1] = __ldcg(q + 1);
+      }
+#pragma unroll
+    for (int t = 0; t < 4; ++t)
+      if (sp0 + t < p.splits) {
+        acc[0] += v[t][0].x;
+        acc[1] += v[t][0].y;
+        acc[2] += v[t][0].z;
+        acc[3] += v[t][0].w;
+        acc[4] += v[t][1].x;
+        acc[5] += v[t][1].y;
+        acc[6] += v[t][1].z;
+        acc[7] += v[t][1].w;
+      }
+  }
+  const float rs = (FMT == 0 ? bf16_bits_to_float(p.scale[n]) : 1.0f) * (p.rotated ? 0.0078125f : 1.0f);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int64_t m = m0 + j;
+    if (m < p.m) __stcs(p.y + m * p.n + n, float_to_bf16_bits_rn(acc[j] * p.xs[m] * rs));
   }
 }
 

@@ -301,47 +301,30 @@ cudaError_t make_tmap_i8(CUtensorMap* map, const void* base, int64_t rows, int64
 }
 
 // Split-K workspace, one per device, made on the first split launch there:
-// fp32 partial tiles and per-tile arrival counters (zeroed once; the last
-// unit of every tile resets its counter).
-constexpr size_t kTcWsBytes = size_t(32) << 20;
-constexpr int64_t kTcMaxCounters = 8192;
-struct TcWorkspace {
-  float* ws = nullptr;
-  int* counters = nullptr;
-};
-TcWorkspace g_tc_ws[kMaxDevices];
+// the fp32 partial tiles of the units.
+constexpr size_t kTcWsBytes = size_t(16) << 20;
+float* g_tc_ws[kMaxDevices];
 std::mutex g_tc_ws_mu;
 
-cudaError_t tc_workspace(TcWorkspace* out) {
+cudaError_t tc_workspace(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_tc_ws_mu);
-  TcWorkspace& w = g_tc_ws[dev];
-  if (w.ws == nullptr) {
+  if (g_tc_ws[dev] == nullptr) {
     void* a = nullptr;
-    void* c = nullptr;
     e = cudaMalloc(&a, kTcWsBytes);
     if (e != cudaSuccess) return e;
-    e = cudaMalloc(&c, kTcMaxCounters * sizeof(int));
-    if (e == cudaSuccess) e = cudaMemset(c, 0, kTcMaxCounters * sizeof(int));
-    if (e == cudaSuccess) e = cudaDeviceSynchronize();
-    if (e != cudaSuccess) {
-      cudaFree(a);
-      if (c) cudaFree(c);
-      return e;
-    }
-    w.ws = static_cast<float*>(a);
-    w.counters = static_cast<int*>(c);
+    g_tc_ws[dev] = static_cast<float*>(a);
   }
-  *out = w;
+  *out = g_tc_ws[dev];
   return cudaSuccess;
 }
 
 // Cost, in scale blocks, of the busiest CTA when `units` units of a tile
 // split S ways are dealt round-robin to min(sms, units) persistent CTAs;
-// a split unit also pays about one block for its partial tile.
+// a split unit also pays about half a block for its partial tile.
 double tc_split_cost(int64_t tiles, int ng, int S, int sms) {
   const int64_t units = tiles * S;
   const int64_t grid = std::min<int64_t>(sms, units);
@@ -350,11 +333,26 @@ double tc_split_cost(int64_t tiles, int ng, int S, int sms) {
     double t = 0.0;
     for (int64_t u = c; u < units; u += grid) {
       const int64_t sp = u % S;
-      t += static_cast<double>((sp + 1) * ng / S - sp * ng / S) + 0.25 + (S > 1 ? 1.0 : 0.0);
+      t += static_cast<double>((sp + 1) * ng / S - sp * ng / S) + 0.25 + (S > 1 ? 0.5 : 0.0);
     }
     worst = std::max(worst, t);
   }
   return worst;
+}
+
+// A launch that may begin while the stream's previous kernel drains (the
+// kernel waits for it before reading that kernel's outputs).
+cudaLaunchConfig_t pdl_config(dim3 grid, dim3 block, size_t smem, cudaStream_t stream, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
 }
 
 template <int FMT, bool PARTIALS, int BMAX>
@@ -364,8 +362,14 @@ cudaError_t launch_tc_t(const CUtensorMap& tw, const CUtensorMap& tx, const TcPa
   static std::atomic<int> configured[kMaxDevices];
   cudaError_t e = ensure_smem(kernel, kTcSmemBytes, configured);
   if (e != cudaSuccess) return e;
-  kernel<<<grid, kTcThreads, kTcSmemBytes, stream>>>(tw, tx, p);
-  return cudaGetLastError();
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pdl_config(dim3(grid), dim3(kTcThreads), kTcSmemBytes, stream, attr);
+  e = cudaLaunchKernelEx(&cfg, kernel, tw, tx, p);
+  if (e != cudaSuccess || p.splits <= 1) return e;
+  const int64_t threads = p.tiles * kTcBN * (p.bm / 8);
+  cudaLaunchConfig_t rcfg = pdl_config(dim3(static_cast<unsigned>((threads + kTcReduceThreads - 1) / kTcReduceThreads)),
+                                       dim3(kTcReduceThreads), 0, stream, attr);
+  return cudaLaunchKernelEx(&rcfg, tc_split_reduce_kernel<FMT>, p);
 }
 
 }  // namespace
@@ -409,7 +413,7 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream) {
   // split K when there are too few tiles to fill the SMs
   const int ng = static_cast<int>(a.k / (a.fmt == 0 ? kGroupTrunk : kGroupHead));
   p.splits = 1;
-  if (p.bm <= kTcSplitMaxBM && p.tiles <= kTcMaxCounters && a.partials == nullptr) {
+  if (p.bm <= kTcSplitMaxBM && a.partials == nullptr) {
     double best = tc_split_cost(p.tiles, ng, 1, d.num_sms);
     for (int S = 2; S <= std::min(ng, 32); ++S) {
       if (static_cast<size_t>(p.tiles) * S * p.bm * kTcBN * sizeof(float) > kTcWsBytes) break;
@@ -422,11 +426,8 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream) {
   }
   p.units = p.tiles * p.splits;
   if (p.splits > 1) {
-    TcWorkspace w;
-    e = tc_workspace(&w);
+    e = tc_workspace(&p.ws);
     if (e != cudaSuccess) return e;
-    p.ws = w.ws;
-    p.counters = w.counters;
   }
   p.xs = a.xs;
   p.sub = a.sub;
@@ -444,6 +445,13 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   const int grid = static_cast<int>(std::min<int64_t>(d.num_sms, p.units));
   const bool part = a.partials != nullptr;
+  if (p.bm <= 32) {
+    if (a.fmt == 0)
+      return part ? launch_tc_t<0, true, 32>(tw, tx, p, grid, stream)
+                  : launch_tc_t<0, false, 32>(tw, tx, p, grid, stream);
+    return part ? launch_tc_t<1, true, 32>(tw, tx, p, grid, stream)
+                : launch_tc_t<1, false, 32>(tw, tx, p, grid, stream);
+  }
   if (p.bm <= kTcSplitMaxBM) {
     if (a.fmt == 0)
       return part ? launch_tc_t<0, true, kTcSplitMaxBM>(tw, tx, p, grid, stream)
