@@ -135,7 +135,16 @@ iq8r_status iq8r_rotate_quant_act(const uint16_t* x_bf16, int64_t m, int64_t k, 
  * with P the exact int32 dot product of the codes over block g (256 or 128
  * of K); /128 only when w->rotated. The sum over g is carried in fp32 or
  * exact integers, so y matches the float64 value to within its bf16
- * rounding plus ~1e-6 of the output's scale. */
+ * rounding plus ~1e-6 of the output's scale.
+ * Kernels: m <= 8 streams the weights through the GEMV; larger m runs the
+ * tensor-core GEMM. When the GEMM has fewer output tiles than SMs it splits
+ * K: the fp32 partial tiles go to a per-device workspace (16 MiB, allocated
+ * by the first such call on the device and kept for the process, so make
+ * that first call before any stream capture) and a second kernel adds them
+ * in a fixed order, so the result does not depend on timing. Calls on
+ * different streams that both split K and overlap in time share that
+ * workspace and race; order them on one stream. Results are the same bits
+ * from call to call. */
 iq8r_status iq8r_linear(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,
                         uint16_t* y_bf16, cudaStream_t stream);
 
