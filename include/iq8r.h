@@ -168,6 +168,25 @@ iq8r_status iq8r_linear_bf16(const uint16_t* x_bf16, int64_t m, const iq8r_weigh
 iq8r_status iq8r_linear_ex(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,
                            uint16_t* y_bf16, int32_t path, cudaStream_t stream);
 
+/* iq8r_linear that allocates nothing (no counterpart on the pages; an
+ * interface for callers that must not allocate, e.g. inside their own
+ * memory pools or graphs). Same arguments, same kernel choice and same
+ * split plan as iq8r_linear, so y is the same bits; but the split-K partial
+ * tiles go to a fixed array of 8 MiB in the library's own device image
+ * instead of an allocated workspace.
+ *   - Set-up: the first call on a device looks up that array's address
+ *     (cudaGetSymbolAddress) and sets kernel attributes; make it before any
+ *     stream capture. No call allocates or frees device memory.
+ *   - A call whose split plan needs more than 8 MiB of partial tiles
+ *     (units x 128 x tokens-per-tile x 4 bytes) returns
+ *     IQ8R_ERR_UNSUPPORTED and launches nothing; iq8r_linear handles it.
+ *   - Nothing in the array needs to start at zero: every partial tile is
+ *     written in full before the second pass reads it.
+ *   - There is one array per device: calls that overlap in time (different
+ *     streams, or other threads) race on it; order them on one stream. */
+iq8r_status iq8r_linear_noalloc(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,
+                                uint16_t* y_bf16, cudaStream_t stream);
+
 /* Debug twin of iq8r_linear: writes the exact per-block int32 partial sums
  * P[i][j][g] = sum_{k in block g} xq[i][k] * codes[n0 + j][k] for rows
  * n0 <= n < n1 instead of y, computed by the same kernel code as the

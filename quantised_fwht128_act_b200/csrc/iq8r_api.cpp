@@ -75,8 +75,10 @@ iq8r::LinearArgs make_args(const int8_t* xq, const float* xs, int64_t m, const i
   return a;
 }
 
-// Choose and launch a kernel for y or partials.
-iq8r_status run_linear(const iq8r::LinearArgs& a, int32_t path, const char* fn, cudaStream_t stream) {
+// Choose and launch a kernel for y or partials. fixed_scratch: the
+// no-allocation variant (split-K scratch from the static array).
+iq8r_status run_linear(const iq8r::LinearArgs& a, int32_t path, const char* fn, cudaStream_t stream,
+                       bool fixed_scratch = false) {
   if (path != IQ8R_PATH_AUTO && path != IQ8R_PATH_GEMV && path != IQ8R_PATH_TC)
     return fail(IQ8R_ERR_INVALID_ARG, "%s: unknown path %d", fn, path);
   if (a.m == 0) return ok();
@@ -94,9 +96,26 @@ iq8r_status run_linear(const iq8r::LinearArgs& a, int32_t path, const char* fn, 
     else
       return fail(IQ8R_ERR_UNSUPPORTED, "%s: %s", fn, why.c_str());
   }
-  const cudaError_t e = use_tc ? iq8r::launch_gemm_tc(a, stream) : iq8r::launch_gemv(a, stream);
+  bool too_big = false;
+  const cudaError_t e = use_tc ? iq8r::launch_gemm_tc(a, stream, fixed_scratch, &too_big) : iq8r::launch_gemv(a, stream);
   if (e != cudaSuccess) return cuda_fail(e, fn);
+  if (too_big)
+    return fail(IQ8R_ERR_UNSUPPORTED, "%s: the split-K plan needs more scratch than the fixed array holds", fn);
   return ok();
+}
+
+// y for iq8r_linear / iq8r_linear_ex / iq8r_linear_noalloc.
+iq8r_status linear_y(const char* fn, const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,
+                     uint16_t* y_bf16, int32_t path, cudaStream_t stream, bool fixed_scratch) {
+  iq8r_status st = check_weight(w, fn);
+  if (st != IQ8R_OK) return st;
+  if (m < 0 || m > kMaxGridRows) return fail(IQ8R_ERR_INVALID_ARG, "%s: m = %lld out of range", fn, (long long)m);
+  if (m == 0) return ok();
+  if (!xq || !x_scale || !y_bf16) return fail(IQ8R_ERR_INVALID_ARG, "%s: NULL buffer", fn);
+  if (!aligned16(xq) || !aligned16(y_bf16)) return fail(IQ8R_ERR_INVALID_ARG, "%s: xq and y must be 16-byte aligned", fn);
+  iq8r::LinearArgs a = make_args(xq, x_scale, m, w);
+  a.y = y_bf16;
+  return run_linear(a, path, fn, stream, fixed_scratch);
 }
 
 }  // namespace
@@ -161,16 +180,12 @@ iq8r_status iq8r_rotate_quant_act(const uint16_t* x_bf16, int64_t m, int64_t k, 
 
 iq8r_status iq8r_linear_ex(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w, uint16_t* y_bf16,
                            int32_t path, cudaStream_t stream) {
-  const char* fn = "iq8r_linear";
-  iq8r_status st = check_weight(w, fn);
-  if (st != IQ8R_OK) return st;
-  if (m < 0 || m > kMaxGridRows) return fail(IQ8R_ERR_INVALID_ARG, "%s: m = %lld out of range", fn, (long long)m);
-  if (m == 0) return ok();
-  if (!xq || !x_scale || !y_bf16) return fail(IQ8R_ERR_INVALID_ARG, "%s: NULL buffer", fn);
-  if (!aligned16(xq) || !aligned16(y_bf16)) return fail(IQ8R_ERR_INVALID_ARG, "%s: xq and y must be 16-byte aligned", fn);
-  iq8r::LinearArgs a = make_args(xq, x_scale, m, w);
-  a.y = y_bf16;
-  return run_linear(a, path, fn, stream);
+  return linear_y("iq8r_linear", xq, x_scale, m, w, y_bf16, path, stream, false);
+}
+
+iq8r_status iq8r_linear_noalloc(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,
+                                uint16_t* y_bf16, cudaStream_t stream) {
+  return linear_y("iq8r_linear_noalloc", xq, x_scale, m, w, y_bf16, IQ8R_PATH_AUTO, stream, true);
 }
 
 iq8r_status iq8r_linear_bf16(const uint16_t* x_bf16, int64_t m, const iq8r_weight* w, uint16_t* y_bf16,

@@ -52,7 +52,10 @@ cudaError_t launch_act_quant(const uint16_t* x, int64_t m, int64_t k, int rotate
                              float* xs, cudaStream_t stream);
 cudaError_t launch_gemv(const LinearArgs& a, cudaStream_t stream);
 bool gemv_supported(int64_t k, std::string* why);
-cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream);
+// fixed_scratch: split-K partials go to the static no-allocation array; a
+// plan that needs more than it holds sets *too_big and launches nothing.
+cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_scratch = false,
+                           bool* too_big = nullptr);
 bool gemm_tc_supported(const LinearArgs& a, std::string* why);
 cudaError_t read_and_clear_device_error(uint32_t* err);
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream);

@@ -322,6 +322,30 @@ cudaError_t tc_workspace(float** out) {
   return cudaSuccess;
 }
 
+// Fixed scratch of the no-allocation entry point: split-K partial tiles in a
+// static device array (part of the module image, so nothing is allocated at
+// call time). Its address is looked up once per device.
+constexpr size_t kNoAllocWsBytes = size_t(8) << 20;
+static __device__ __align__(256) float g_noalloc_ws[kNoAllocWsBytes / sizeof(float)];
+float* g_noalloc_ptr[kMaxDevices];
+std::atomic<int> g_noalloc_ready[kMaxDevices];
+
+cudaError_t noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  if (g_noalloc_ready[dev].load(std::memory_order_acquire) == 0) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_noalloc_ws);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = static_cast<float*>(ptr);
+    g_noalloc_ready[dev].store(1, std::memory_order_release);
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
 // Cost, in scale blocks, of the busiest CTA when `units` units of a tile
 // split S ways are dealt round-robin to min(sms, units) persistent CTAs;
 // a split unit also pays about half a block for its partial tile.
@@ -391,7 +415,8 @@ bool gemm_tc_supported(const LinearArgs& a, std::string* why) {
   return true;
 }
 
-cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream) {
+cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_scratch, bool* too_big) {
+  if (too_big) *too_big = false;
   if (a.m == 0 || a.n == 0) return cudaSuccess;
   DeviceInfo d;
   cudaError_t e = device_info(&d);
@@ -426,7 +451,18 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream) {
   }
   p.units = p.tiles * p.splits;
   if (p.splits > 1) {
-    e = tc_workspace(&p.ws);
+    if (fixed_scratch) {
+      // the same plan as the allocating path; refuse it if the fixed array
+      // cannot hold its partial tiles (nothing is launched)
+      const size_t need = static_cast<size_t>(p.units) * kTcBN * p.bm * sizeof(float);
+      if (need > kNoAllocWsBytes) {
+        if (too_big) *too_big = true;
+        return cudaSuccess;
+      }
+      e = noalloc_scratch(&p.ws);
+    } else {
+      e = tc_workspace(&p.ws);
+    }
     if (e != cudaSuccess) return e;
   }
   p.xs = a.xs;
