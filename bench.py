@@ -81,14 +81,45 @@ def fused_bytes(m, k, n, fmt):
     return linear_bytes(m, k, n, fmt) - m * k - 4 * m + 2 * m * k
 
 
+# iq8r_linear_bf16 is one launch (activation quantiser fused into the GEMV)
+# for M <= 8 with M * K <= 16384; iq8r_linear picks the GEMV for M <= 2
+# (both as documented in include/iq8r.h)
+FUSE_MAX_M, FUSE_MAX_ELEMS, GEMV_MAX_M = 8, 16384, 2
+
+
+def one_launch(m, k):
+    return m <= FUSE_MAX_M and m * k <= FUSE_MAX_ELEMS
+
+
 def step_bytes(m, k, n, fmt, fused=None):
-    """Algorithmic bytes of one step: the fused layer (one launch, M <= 8),
-    else the activation kernel plus the linear."""
+    """Algorithmic bytes of one step: the fused layer (one launch), else the
+    activation kernel plus the linear."""
     if fused is None:
-        fused = m <= 8
+        fused = one_launch(m, k)
     if fused:
         return fused_bytes(m, k, n, fmt)
     return act_bytes(m, k) + linear_bytes(m, k, n, fmt)
+
+
+def graph_kernel_nodes(g):
+    """Kernel nodes in a captured torch CUDA graph (None if it cannot be
+    inspected)."""
+    if g is None:
+        return 0
+    try:
+        from cuda.bindings import runtime as rt
+        h = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+        err, _, num = rt.cudaGraphGetNodes(h, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, num = rt.cudaGraphGetNodes(h, num)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kinds = [rt.cudaGraphNodeGetType(nd) for nd in nodes[:num]]
+        return sum(1 for e, t in kinds if e == rt.cudaError_t.cudaSuccess
+                   and t == rt.cudaGraphNodeType.cudaGraphNodeTypeKernel)
+    except Exception:
+        return None
 
 
 def max_over_ranks(ms, world, device):
@@ -114,7 +145,7 @@ def is_hbm_bound(m, k, n, fmt, fused=None):
     the tensor cores above it. Decode and verify steps are HBM-bound and are
     reported in GB/s; prefill is tensor-bound and reported in int8 TOPS."""
     if fused is None:
-        fused = m <= 8
+        fused = one_launch(m, k)
     hbm, bf16_tf, _ = peaks()
     lin_b = fused_bytes(m, k, n, fmt) if fused else linear_bytes(m, k, n, fmt)
     return 2.0 * m * n * k / lin_b < bf16_tf * INT8_OVER_BF16 * 1e12 / (hbm * 1e9)
@@ -221,11 +252,12 @@ class ClockSampler:
 
 # ------------------------------------------------------------- workload
 
-def make_inputs(cfg_name, copies_hint=None):
+def make_inputs(cfg_name, m_override=None):
     """Host inputs: x copies (bf16 bits) and the packed weight (host packer)."""
     import quantised_fwht128_act_b200 as iq8r
     from iq8r_inputs import WORKLOADS, f32_to_bf16_bits, gen_act, gen_workload
     m, k, n, fmt, _ = CONFIGS[cfg_name]
+    m = m_override or m
     wl = WORKLOADS.get(cfg_name, WORKLOADS["decode"])
     x0, w = gen_workload(wl, m=m, n=n, k=k)
     packed = iq8r.iq8r_pack(w, fmt, True)
@@ -241,8 +273,9 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
     m, k, n, fmt, _ = CONFIGS[args.config]
+    m = getattr(args, "m", None) or m
     K, W = args.steps, args.warmup
-    x0, (codes, sub, scale), wl = make_inputs(args.config)
+    x0, (codes, sub, scale), wl = make_inputs(args.config, m)
 
     # rotating copies so that consecutive uses of one copy are > 3x L2 apart
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -262,12 +295,10 @@ def run_ours(args, rank, world, local_rank):
     xsc = [torch.empty((m,), dtype=torch.float32, device=dev) for _ in range(R)]
     y = [torch.empty((m, n), dtype=torch.bfloat16, device=dev) for _ in range(R)]
     path = {"auto": iq8r.IQ8R_PATH_AUTO, "gemv": iq8r.IQ8R_PATH_GEMV, "tc": iq8r.IQ8R_PATH_TC}[args.path]
-    fused = m <= 8 and args.path == "auto"  # one launch: the GEMV rotates and quantises x itself
+    fused = one_launch(m, k) and args.path == "auto"  # the GEMV rotates and quantises x itself
 
     def linear(r):
         iq8r.iq8r_linear_ex(xq[r], xsc[r], weights[r], y[r], path=path)
-
-    launches_per_step = 1 if fused else 2  # else the activation kernel + the tensor-core GEMM
 
     def step(j):
         r = j % R
@@ -294,7 +325,10 @@ def run_ours(args, rank, world, local_rank):
     n_main, tail = divmod(K, C)
 
     def capture(nsteps, offset):
-        g = torch.cuda.CUDAGraph()
+        try:
+            g = torch.cuda.CUDAGraph(keep_graph=True)  # kept so its kernel nodes can be counted
+        except TypeError:
+            g = torch.cuda.CUDAGraph()
         evs = None if fused else [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
                                   for _ in range(nsteps)]
         with torch.cuda.graph(g, stream=stream):
@@ -308,10 +342,16 @@ def run_ours(args, rank, world, local_rank):
                 evs[j][1].record()
                 linear(r)
                 evs[j][2].record()
+        g.instantiate()
         return g, evs
 
     g_main, ev_main = capture(C, 0) if n_main else (None, None)
     g_tail, ev_tail = capture(tail, 0) if tail else (None, None)
+    # this library's kernel launches inside the timed region: the kernel
+    # nodes of each captured graph times its replays
+    counts = [graph_kernel_nodes(g) for g in (g_main, g_tail)]
+    gpu_launches = (None if any(c is None for c, g in zip(counts, (g_main, g_tail)) if g is not None)
+                    else n_main * (counts[0] or 0) + (counts[1] or 0))
     # one untimed replay of each graph (upload, first-touch)
     for g in (g_main, g_tail):
         if g is not None:
@@ -410,7 +450,7 @@ def run_ours(args, rank, world, local_rank):
     # the kernel's bound: HBM below the ridge point (int8 ops per byte at
     # which the tensor peak and the HBM peak take equal time), tensor above
     hbm_bound = is_hbm_bound(m, k, n, fmt, fused)
-    on_tc = args.path == "tc" or (args.path == "auto" and m > 8)
+    on_tc = args.path == "tc" or (args.path == "auto" and not fused and m > GEMV_MAX_M)
     kname = ("gemv_kernel (fused act, one launch per step)" if fused else
              "gemm_tc_kernel (tcgen05 kind::i8)" if on_tc else "gemv_kernel")
     kfiles = ["gemm_tc.cuh", "iq8r_device.cuh"] if on_tc else ["gemv.cuh", "act_quant.cuh", "iq8r_device.cuh"]
@@ -463,7 +503,7 @@ def run_ours(args, rank, world, local_rank):
                              "CUDA graphs of the K steps; events inside the graphs time each kernel"},
         "roofline": roof,
         "clocks": clocks,
-        "gpu_launches": launches_per_step * K,
+        "gpu_launches": gpu_launches,
         "e2e": e2e,
         "cpu_baseline": None,
     }
@@ -518,7 +558,7 @@ def run_oracle(cfg_name, budget_s, steps=None):
         oracle.linear(q, a, fmt, *packed, rotated=True)
     dt = time.perf_counter() - t
     if is_hbm_bound(m, k, n, fmt):
-        b = step_bytes(m_s, k, n_s, fmt, fused=m <= 8)
+        b = step_bytes(m_s, k, n_s, fmt, fused=one_launch(m, k))
         value, unit, what = b * reps / dt / 1e9, "GB/s", "algorithmic bytes"
     else:
         value, unit, what = 2.0 * m_s * n_s * k * reps / dt / 1e12, "TOPS", "int8 ops (2 M N K)"
@@ -556,6 +596,7 @@ def main(argv=None):
     ap.add_argument("--config", choices=sorted(CONFIGS), default="decode")
     ap.add_argument("--path", choices=["auto", "gemv", "tc"], default="auto",
                     help="force the linear's kernel (auto: the library's choice)")
+    ap.add_argument("--m", type=int, default=None, help="override the workload's token count M")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill TOPS line of the decode run")

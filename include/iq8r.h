@@ -136,8 +136,9 @@ iq8r_status iq8r_rotate_quant_act(const uint16_t* x_bf16, int64_t m, int64_t k, 
  * of K); /128 only when w->rotated. The sum over g is carried in fp32 or
  * exact integers, so y matches the float64 value to within its bf16
  * rounding plus ~1e-6 of the output's scale.
- * Kernels: m <= 8 streams the weights through the GEMV; larger m runs the
- * tensor-core GEMM. When the GEMM has fewer output tiles than SMs it splits
+ * Kernels: m <= 2 streams the weights through the GEMV; larger m runs the
+ * tensor-core GEMM (measured on B200: from 3 tokens on it is as fast or
+ * faster, at every workload shape). When the GEMM has fewer output tiles than SMs it splits
  * K: the fp32 partial tiles go to a per-device workspace (16 MiB, allocated
  * by the first such call on the device and kept for the process, so make
  * that first call before any stream capture) and a second kernel adds them
@@ -151,10 +152,11 @@ iq8r_status iq8r_linear(const int8_t* xq, const float* x_scale, int64_t m, const
 /* The whole layer from bf16 activations: rotate + quantise x (as
  * iq8r_rotate_quant_act, rotating iff w->rotated) and then iq8r_linear.
  * For m <= 8 and m * k <= 16384 (a decode step), or when xq_out and
- * x_scale_out are not given, this is one kernel: every CTA of the
- * weight-streaming GEMV rotates and quantises x itself while its first
+ * x_scale_out are not given (m <= 8 only), this is one kernel: every CTA of
+ * the weight-streaming GEMV rotates and quantises x itself while its first
  * weight tiles stream in. Otherwise the codes are staged in xq_out /
- * x_scale_out and a second kernel consumes them.
+ * x_scale_out and iq8r_linear consumes them; give the staging buffers for
+ * long K (a verify block), where that is the faster way.
  *   x_bf16      device bf16 [m][w->k], 16-byte aligned (w->k % 128 == 0)
  *   y_bf16      device bf16 [m][w->n] (out), 16-byte aligned
  *   xq_out      device int8 [m][w->k] (out) or NULL: the activation codes

@@ -40,7 +40,7 @@ constexpr int64_t kMaxGridRows = (int64_t(1) << 31) - 1;
 // many activation elements (M * K); beyond it two launches are cheaper.
 constexpr int64_t kFuseMaxElems = 16384;
 // Above this many tokens the automatic choice is the tensor-core GEMM.
-constexpr int64_t kGemvMaxM = 8;
+constexpr int64_t kGemvMaxM = 2;
 
 iq8r_status check_weight(const iq8r_weight* w, const char* fn) {
   if (!w) return fail(IQ8R_ERR_INVALID_ARG, "%s: weight is NULL", fn);

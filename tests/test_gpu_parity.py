@@ -118,11 +118,15 @@ def test_partials_bit_exact_workloads(name):
     assert np.array_equal(gpu_partials(x, W), oracle.partials(xq, codes, g))
 
 
-@pytest.mark.parametrize("m,n,k", [(3, 1000, 768), (5, 37, 2304), (13, 64, 512), (2, 9, 4352), (8, 20, 256)])
-def test_partials_bit_exact_ragged(m, n, k):
+# the GEMV forced (every token-tile width 1..8), and the library's own choice
+@pytest.mark.parametrize("path", ["gemv", "auto"])
+@pytest.mark.parametrize("m,n,k", [(3, 1000, 768), (5, 37, 2304), (13, 64, 512), (2, 9, 4352), (8, 20, 256),
+                                   (7, 300, 1024), (4, 129, 2560)])
+def test_partials_bit_exact_ragged(m, n, k, path):
     x, _, _, (codes, _, _), W = case("decode", m=m, n=n, k=k, seed=7 + m + n + k)
     xq, _ = oracle.act_quant(x)
-    assert np.array_equal(gpu_partials(x, W), oracle.partials(xq, codes, 256))
+    p = iq8r.IQ8R_PATH_GEMV if path == "gemv" else iq8r.IQ8R_PATH_AUTO
+    assert np.array_equal(gpu_partials(x, W, path=p), oracle.partials(xq, codes, 256))
 
 
 def test_partials_lm_head_windows():
@@ -172,17 +176,22 @@ def test_linear_within_tolerance_workloads(name):
     assert st["bit_equal_frac"] > 0.99
 
 
-@pytest.mark.parametrize("m,n,k", [(1, 1000, 768), (3, 37, 2304), (13, 64, 512), (5, 9, 4352), (2, 333, 1280)])
-def test_linear_within_tolerance_ragged(m, n, k):
+@pytest.mark.parametrize("path", ["gemv", "auto"])
+@pytest.mark.parametrize("m,n,k", [(1, 1000, 768), (3, 37, 2304), (13, 64, 512), (5, 9, 4352), (2, 333, 1280),
+                                   (8, 77, 1536)])
+def test_linear_within_tolerance_ragged(m, n, k, path):
     x, _, fmt, packed, W = case("decode", m=m, n=n, k=k, seed=11 + m + n + k)
     y64 = oracle_linear(x, fmt, packed)
-    check_output(gpu_linear(x, W), y64, oracle.linear_bf16(y64))
+    p = iq8r.IQ8R_PATH_GEMV if path == "gemv" else iq8r.IQ8R_PATH_AUTO
+    check_output(gpu_linear(x, W, path=p), y64, oracle.linear_bf16(y64))
 
 
-def test_linear_lm_head_small():
+@pytest.mark.parametrize("path", ["gemv", "auto"])
+def test_linear_lm_head_small(path):
     x, _, fmt, packed, W = case("lm_head8", m=8, n=2000, k=5120, seed=45)
     y64 = oracle_linear(x, fmt, packed)
-    check_output(gpu_linear(x, W), y64, oracle.linear_bf16(y64))
+    p = iq8r.IQ8R_PATH_GEMV if path == "gemv" else iq8r.IQ8R_PATH_AUTO
+    check_output(gpu_linear(x, W, path=p), y64, oracle.linear_bf16(y64))
 
 
 def test_linear_unrotated_weight():
@@ -285,7 +294,11 @@ def test_linear_bf16_fused_matches_two_call_path(name, m, n, k):
     q, a = oracle.act_quant(x)
     assert np.array_equal(xq_out.cpu().numpy(), q)
     assert np.array_equal(xs_out.cpu().numpy().view(np.uint32), a.view(np.uint32))
-    y2 = gpu_linear(x, W)
+    # one launch (the GEMV with the quantiser fused) when m * k <= 16384, else
+    # the activation kernel and iq8r_linear's own choice: the same arithmetic
+    # as the two-call path through that kernel
+    fused = x.shape[0] * x.shape[1] <= 16384
+    y2 = gpu_linear(x, W, path=iq8r.IQ8R_PATH_GEMV if fused else iq8r.IQ8R_PATH_AUTO)
     assert np.array_equal(host_bits(y), y2)
     y64 = oracle_linear(x, fmt, packed)
     check_output(host_bits(y), y64, oracle.linear_bf16(y64))
