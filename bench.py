@@ -82,13 +82,13 @@ def fused_bytes(m, k, n, fmt):
 
 
 # iq8r_linear_bf16 is one launch (activation quantiser fused into the GEMV)
-# for M <= 8 with M * K <= 16384; iq8r_linear picks the GEMV for M <= 2
-# (both as documented in include/iq8r.h)
+# for M <= 2 and for M <= 8 with M * K <= 16384; iq8r_linear picks the GEMV
+# for M <= 2 (both as documented in include/iq8r.h)
 FUSE_MAX_M, FUSE_MAX_ELEMS, GEMV_MAX_M = 8, 16384, 2
 
 
 def one_launch(m, k):
-    return m <= FUSE_MAX_M and m * k <= FUSE_MAX_ELEMS
+    return m <= GEMV_MAX_M or (m <= FUSE_MAX_M and m * k <= FUSE_MAX_ELEMS)
 
 
 def step_bytes(m, k, n, fmt, fused=None):

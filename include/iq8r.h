@@ -151,7 +151,7 @@ iq8r_status iq8r_linear(const int8_t* xq, const float* x_scale, int64_t m, const
 
 /* The whole layer from bf16 activations: rotate + quantise x (as
  * iq8r_rotate_quant_act, rotating iff w->rotated) and then iq8r_linear.
- * For m <= 8 and m * k <= 16384 (a decode step), or when xq_out and
+ * For m <= 2, for m <= 8 with m * k <= 16384, and when xq_out and
  * x_scale_out are not given (m <= 8 only), this is one kernel: every CTA of
  * the weight-streaming GEMV rotates and quantises x itself while its first
  * weight tiles stream in. Otherwise the codes are staged in xq_out /

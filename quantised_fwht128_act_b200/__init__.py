@@ -254,7 +254,8 @@ def iq8r_linear(xq, x_scale, weight: IQ8RWeight, y=None, stream=None):
 
 def iq8r_linear_bf16(x, weight: IQ8RWeight, y=None, xq_out=None, x_scale_out=None, stream=None):
     """y = x W^T from bf16 activations [M, K] (rotated and quantised inside;
-    one launch for M <= 8 with M * K <= 16384). xq_out / x_scale_out receive
+    one launch for M <= 2, and for M <= 8 with M * K <= 16384). xq_out /
+    x_scale_out receive
     the activation codes and scales; staging buffers are made here when the
     call is not a one-launch decode step and none are given."""
     import torch
@@ -263,7 +264,7 @@ def iq8r_linear_bf16(x, weight: IQ8RWeight, y=None, xq_out=None, x_scale_out=Non
     m = x.shape[0]
     if y is None:
         y = torch.empty((m, weight.n), dtype=torch.bfloat16, device=x.device)
-    if m > 8 or m * weight.k > 16384:
+    if m > 8 or (m > 2 and m * weight.k > 16384):
         if xq_out is None:
             xq_out = torch.empty((m, weight.k), dtype=torch.int8, device=x.device)
         if x_scale_out is None:

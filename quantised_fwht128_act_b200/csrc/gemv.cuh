@@ -63,6 +63,9 @@ struct GemvPlan {
   int stage_bytes;  // codes + scales of one stage, 128-aligned
   int sc_off;       // offset of the scales within a stage
   int s2_off;       // offset of the trunk's row scales within a stage
+  int pre;          // trunk: 1 = the CTA's row scales are loaded once, up front
+  int pre_s1;       // pre: bytes of the sub-scale window in shared memory
+  int pre_bytes;    // pre: sub-scale window + row-scale window
   int smem;         // total dynamic shared memory
 };
 
@@ -85,7 +88,7 @@ __host__ __device__ inline GemvPlan gemv_plan_for(int mt, int fmt, int k, int rt
   p.s2_off = p.sc_off + gemv_s1_window(rt, kc);
   p.stage_bytes = gemv_align128(p.sc_off + gemv_sc_bytes(fmt, rt, kc));
   // [act MT*K][warps x depth stages][barriers: warps x depth + 1][counter]
-  p.smem = gemv_align128(mt * k) + warps * depth * p.stage_bytes + 8 * (warps * depth + 1) + 16;
+  p.smem = gemv_align128(mt * k) + warps * depth * p.stage_bytes + 8 * (warps * depth + 2) + 16;
   return p;
 }
 
@@ -153,6 +156,41 @@ __device__ __forceinline__ void gemv_fused_act(const LinearArgs& a, int8_t* act,
   const int warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
   const int iters = (slots + blockDim.x - 1) / blockDim.x;
+  if (MT <= 2 && iters == 1) {
+    // every thread holds at most one slot per token: one load and one
+    // transform, kept in registers across the CTA-wide amax
+    float v[MT][kActSlot];
+    float mx1[MT];
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      mx1[m] = 0.0f;
+      const int s = threadIdx.x;
+      if (m < M && s < slots) {
+        act_load_slot(a.x + static_cast<int64_t>(m) * K + s * kActSlot, v[m], false);
+      } else {
+#pragma unroll
+        for (int i = 0; i < kActSlot; ++i) v[m][i] = 0.0f;
+      }
+      if (a.rotated) act_fwht_slot(v[m], lane);
+      mx1[m] = act_slot_absmax(v[m]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx1[m] = fmaxf(mx1[m], __shfl_xor_sync(0xffffffffu, mx1[m], o));
+      if (lane == 0) red[m * 32 + warp] = mx1[m];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int m = 0; m < MT; ++m) {
+      if (m >= M) {
+        xscale[m] = 0.0f;
+        continue;
+      }
+      float amax = 0.0f;
+      for (int w = 0; w < nwarps; ++w) amax = fmaxf(amax, red[m * 32 + w]);
+      const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+      xscale[m] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+      if (static_cast<int>(threadIdx.x) < slots) act_store_slot(act + m * K + threadIdx.x * kActSlot, v[m], inv);
+    }
+  } else {
   float mx[MT];
 #pragma unroll
   for (int m = 0; m < MT; ++m) {
@@ -200,6 +238,7 @@ __device__ __forceinline__ void gemv_fused_act(const LinearArgs& a, int8_t* act,
       if (s < slots) act_store_slot(act + m * K + s * kActSlot, v, inv);
     }
   }
+  }
   __syncthreads();
   if (blockIdx.x == 0) {
     if (a.xq_out) {
@@ -217,6 +256,10 @@ __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
   constexpr int G = FMT == 0 ? kGroupTrunk : kGroupHead;
   constexpr int LPB = G / 16;  // lanes per block within a 512-byte step
   constexpr int kGemvUnroll = gemv_unroll(MT, RG);
+  // one or two tokens, one row at a time: stage rows of up to kRegSteps x 512
+  // bytes are consumed from registers (see below)
+  constexpr bool kRegStage = MT <= 2 && RG == 1;
+  constexpr int kRegSteps = 10;
 
   extern __shared__ __align__(128) uint8_t smem[];
   const int K = static_cast<int>(a.k);
@@ -230,18 +273,35 @@ __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + gemv_align128(MT * K) + p.warps * p.depth * p.stage_bytes);
   uint64_t* full = bars + warp * p.depth;
   uint64_t* actbar = bars + p.warps * p.depth;
-  int* counter = reinterpret_cast<int*>(actbar + 1);
+  uint64_t* prebar = actbar + 1;
+  int* counter = reinterpret_cast<int*>(actbar + 2);
+  // trunk scales of the CTA's rows, when loaded up front: [s1 window][s2 window]
+  uint8_t* pre_sc = smem + p.smem - p.pre_bytes;
 
   const int64_t bid = blockIdx.x;
   const int64_t t0 = bid * tiles_base + (bid < tiles_extra ? bid : tiles_extra);
   const int64_t t1 = t0 + tiles_base + (bid < tiles_extra ? 1 : 0);
   const int nchunks = (K + p.kc - 1) / p.kc;
+  const bool pre = FMT == 0 && !PARTIALS && p.pre;
+  const int64_t crow0 = t0 * p.rt;                          // the CTA's first row
+  const int64_t crow1 = min(t1 * p.rt, N);                  // and one past its last
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < p.warps * p.depth; ++s) mbar_init(&bars[s], 1);
     mbar_init(actbar, 1);
+    mbar_init(prebar, 1);
     *counter = 0;
     fence_barrier_init();
+    if (pre && crow1 > crow0) {
+      // one copy each for the sub-scales and the row scales of all the CTA's
+      // rows (16-byte windows; plain loads only past the arrays' last 16 bytes)
+      const GemvWindow w0 = window_copy_plan(pre_sc, a.sub, N * ng, crow0 * ng, crow1 * ng, true);
+      const GemvWindow w1 = window_copy_plan(pre_sc + p.pre_s1, reinterpret_cast<const uint8_t*>(a.scale), 2 * N,
+                                             2 * crow0, 2 * crow1, true);
+      mbar_arrive_expect_tx(prebar, w0.bytes + w1.bytes);
+      if (w0.bytes) bulk_g2s_default(w0.dst, w0.src, w0.bytes, prebar);
+      if (w1.bytes) bulk_g2s_default(w1.dst, w1.src, w1.bytes, prebar);
+    }
   }
   // token rows past M are zero (their codes never reach an output anyway)
   {
@@ -290,7 +350,7 @@ __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
     uint8_t* st = bufs + b * p.stage_bytes;
     const int cbytes = rows * len;
     GemvWindow w0{nullptr, nullptr, 0u}, w1{nullptr, nullptr, 0u};
-    if (!PARTIALS && lane < 3) {
+    if (!PARTIALS && !pre && lane < 3) {
       const int gb = len / G;
       const int64_t o0 = row0 * ng + chunk * (p.kc / G);  // first scale of the stage, in elements
       if (FMT == 0) {
@@ -339,6 +399,10 @@ __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
     const bool ok = mbar_wait(actbar, 0u, kDevErrGemvFull);
     failed = !__all_sync(0xffffffffu, ok);
   }
+  if (pre && crow1 > crow0 && !failed) {
+    const bool ok = mbar_wait(prebar, 0u, kDevErrGemvFull);
+    failed = !__all_sync(0xffffffffu, ok);
+  }
   const float rot = a.rotated ? 0.0078125f : 1.0f;
 
   // Sums of the row group in flight: int64 (trunk) or fp32 (lm_head). They
@@ -360,10 +424,94 @@ __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
     const int gb = len / G;
     // scales start inside their 16-byte window (see window_copy_plan)
     const int64_t so = row0 * ng + chunk * (p.kc / G);
-    const uint8_t* sc = st + p.sc_off + (FMT == 0 ? (so & 15) : ((2 * so) & 15));
-    const uint16_t* s2p = reinterpret_cast<const uint16_t*>(st + p.s2_off + ((2 * row0) & 15));
+    const uint8_t* sc = pre ? pre_sc + ((crow0 * ng) & 15) + (so - crow0 * ng)
+                            : st + p.sc_off + (FMT == 0 ? (so & 15) : ((2 * so) & 15));
+    const uint16_t* s2p = pre ? reinterpret_cast<const uint16_t*>(pre_sc + p.pre_s1 + ((2 * crow0) & 15)) +
+                                    (row0 - crow0)
+                              : reinterpret_cast<const uint16_t*>(st + p.s2_off + ((2 * row0) & 15));
+    const int sstride = pre ? ng : gb;  // scales per row in the stage (or in the CTA's preloaded rows)
     const int nsteps = (len + 511) / 512;
-    for (int r0 = 0; r0 < rows; r0 += RG) {
+    bool refilled = false;
+    if (kRegStage && rows == 1 && nsteps <= kRegSteps) {
+      // one row (chunk) of at most 5 KB: pull it and its scales into
+      // registers, hand the buffer straight back to the copy engine, then
+      // compute -- the copy of the next tile overlaps this tile's arithmetic
+      int4 wv[kRegSteps];
+      uint32_t scv[kRegSteps];
+#pragma unroll
+      for (int u = 0; u < kRegSteps; ++u) {
+        const int o = u * 512 + lane * 16;
+        const bool vr = u < nsteps && !failed && o < len;
+        wv[u] = vr ? *reinterpret_cast<const int4*>(st + o) : make_int4(0, 0, 0, 0);
+        scv[u] = 0u;
+        if (!PARTIALS && vr)
+          scv[u] = FMT == 0 ? static_cast<uint32_t>(sc[o / G])
+                            : static_cast<uint32_t>(reinterpret_cast<const uint16_t*>(sc)[o / G]);
+      }
+      const uint16_t s2b = (FMT == 0 && !PARTIALS) ? s2p[0] : 0;
+      __syncwarp();
+      uses[b] += 1;
+      if (!failed) {
+        issue(b);
+      } else {
+        issued[b].tile = -1;
+      }
+      refilled = true;
+      if (chunk == 0) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          racc[0][m] = 0;
+          facc[0][m] = 0.0f;
+        }
+      }
+      int acc32[MT];
+#pragma unroll
+      for (int m = 0; m < MT; ++m) acc32[m] = 0;
+#pragma unroll
+      for (int u = 0; u < kRegSteps; ++u) {
+        if (u < nsteps) {
+          const int o = u * 512 + lane * 16;
+          const bool valid = !failed && o < len;
+          const int kk = chunk * p.kc + o;
+#pragma unroll
+          for (int m = 0; m < MT; ++m) {
+            const int4 xv = valid ? *reinterpret_cast<const int4*>(act + m * K + kk) : make_int4(0, 0, 0, 0);
+            int q = dot16(wv[u], xv);
+            if (PARTIALS) {
+#pragma unroll
+              for (int off = 1; off < LPB; off <<= 1) q += __shfl_xor_sync(0xffffffffu, q, off);
+              if (valid && m < M && (lane & (LPB - 1)) == 0)
+                a.partials[(static_cast<int64_t>(m) * N + row0) * ng + kk / G] = q;
+            } else if (FMT == 0) {
+              acc32[m] += static_cast<int>(scv[u]) * q;  // <= 10 steps of 255 * 16 * 127^2 < 2^31
+            } else {
+              facc[0][m] = fmaf(static_cast<float>(q), bf16_bits_to_float(static_cast<uint16_t>(scv[u])), facc[0][m]);
+            }
+          }
+        }
+      }
+#pragma unroll
+      for (int m = 0; m < MT; ++m) racc[0][m] += acc32[m];
+      if (!PARTIALS && chunk == nchunks - 1) {
+#pragma unroll
+        for (int m = 0; m < MT; ++m) {
+          float yv;
+          if (FMT == 0) {
+            long long v = racc[0][m];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+            yv = __ll2float_rn(v) * xscale[m] * bf16_bits_to_float(s2b) * rot;
+          } else {
+            float v = facc[0][m];
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+            yv = v * xscale[m] * rot;
+          }
+          if (lane == m && !failed && m < M) a.y[static_cast<int64_t>(m) * N + row0] = float_to_bf16_bits_rn(yv);
+        }
+      }
+    }
+    for (int r0 = 0; r0 < (refilled ? 0 : rows); r0 += RG) {
       if (chunk == 0) {
 #pragma unroll
         for (int i = 0; i < RG; ++i)
@@ -402,9 +550,9 @@ __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
             sfv[u][i] = 0.0f;
             if (!PARTIALS && vr) {
               if (FMT == 0)
-                s1v[u][i] = sc[rl * gb + o / G];
+                s1v[u][i] = sc[rl * sstride + o / G];
               else
-                sfv[u][i] = bf16_bits_to_float(reinterpret_cast<const uint16_t*>(sc)[rl * gb + o / G]);
+                sfv[u][i] = bf16_bits_to_float(reinterpret_cast<const uint16_t*>(sc)[rl * sstride + o / G]);
             }
           }
         }
@@ -479,12 +627,14 @@ __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
       }
     }
     // the buffer is consumed: refill it (the chunk's data is no longer read)
-    __syncwarp();
-    uses[b] += 1;
-    if (!failed) {
-      issue(b);
-    } else {
-      issued[b].tile = -1;
+    if (!refilled) {
+      __syncwarp();
+      uses[b] += 1;
+      if (!failed) {
+        issue(b);
+      } else {
+        issued[b].tile = -1;
+      }
     }
     b = b + 1 == p.depth ? 0 : b + 1;
     if (failed) {
@@ -497,7 +647,8 @@ __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
       break;
     }
   }
-  if (!FUSED && threadIdx.x == 0) mbar_wait(actbar, 0u, kDevErrGemvDrain);  // the shared copy has landed
+  if (!FUSED && threadIdx.x == 0) mbar_wait(actbar, 0u, kDevErrGemvDrain);  // the shared copies have landed
+  if (pre && crow1 > crow0 && threadIdx.x == 0) mbar_wait(prebar, 0u, kDevErrGemvDrain);
 }
 
 }  // namespace iq8r

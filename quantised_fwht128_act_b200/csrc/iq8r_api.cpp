@@ -204,7 +204,7 @@ iq8r_status iq8r_linear_bf16(const uint16_t* x_bf16, int64_t m, const iq8r_weigh
   // its rotation is cheap, or when there is nowhere to stage the codes.
   const bool small = m * w->k <= kFuseMaxElems;
   const bool staged = xq_out && x_scale_out;
-  if (m <= 8 && (small || !staged) && iq8r::gemv_supported(w->k, &why)) {
+  if (m <= 8 && (small || m <= kGemvMaxM || !staged) && iq8r::gemv_supported(w->k, &why)) {
     // one launch: every CTA rotates and quantises x itself, then streams W
     iq8r::LinearArgs a = make_args(nullptr, nullptr, m, w);
     a.y = y_bf16;

@@ -75,7 +75,10 @@ GemvPlan gemv_choose(int mt, int fmt, int k, const DeviceInfo& d) {
   const int avail = budget - gemv_align128(mt * k) - 8 * (warps * kGemvMaxDepth + 1) - 16;
   if (avail <= 0) return none;
   const int per_warp = avail / warps;
-  for (int target = std::min(16 * 1024, (per_warp / 2) & ~511); target >= 512; target -= 512) {
+  // one or two tokens: a stage holds at most 10 steps of 512 bytes, the
+  // register-staged consumer's limit
+  const int cap = mt <= 2 ? 10 * 512 : 16 * 1024;
+  for (int target = std::min(cap, (per_warp / 2) & ~511); target >= 512; target -= 512) {
     GemvPlan p = gemv_plan(mt, fmt, k, target, 2, warps);
     const int depth = std::min(kGemvMaxDepth, per_warp / p.stage_bytes);
     if (depth < 2) continue;
@@ -86,13 +89,29 @@ GemvPlan gemv_choose(int mt, int fmt, int k, const DeviceInfo& d) {
 }
 
 template <int MT, int RG, int FMT, int MODE>
-cudaError_t launch_gemv_t(const LinearArgs& a, const GemvPlan& p, const DeviceInfo& d, cudaStream_t stream) {
+cudaError_t launch_gemv_t(const LinearArgs& a, const GemvPlan& plan, const DeviceInfo& d, cudaStream_t stream) {
   auto kernel = gemv_kernel<MT, RG, FMT, MODE == kGemvPartials, MODE == kGemvFused>;
+  const int64_t tiles = (a.n + plan.rt - 1) / plan.rt;
+  const int64_t grid = std::min<int64_t>(d.num_sms, tiles);
+  GemvPlan p = plan;
+  if (FMT == 0 && MODE != kGemvPartials) {
+    // the trunk's scales of a CTA's rows are small: load them once, up front,
+    // instead of two more copies with every stage
+    const int64_t rows = (tiles + grid - 1) / grid * p.rt;
+    const int64_t ng = a.k / kGroupTrunk;
+    const int64_t s1b = gemv_align16(static_cast<int>(std::min<int64_t>(rows * ng, 1 << 20)) + 32);
+    const int64_t s2b = gemv_align16(static_cast<int>(std::min<int64_t>(2 * rows, 1 << 20)) + 32);
+    const int64_t base = gemv_align16(p.smem);
+    if (base + s1b + s2b <= d.smem_optin - kSmemReserve) {
+      p.pre = 1;
+      p.pre_s1 = static_cast<int>(s1b);
+      p.pre_bytes = static_cast<int>(s1b + s2b);
+      p.smem = static_cast<int>(base + s1b + s2b);
+    }
+  }
   static std::atomic<int> configured[kMaxDevices];
   cudaError_t e = ensure_smem(kernel, p.smem, configured);
   if (e != cudaSuccess) return e;
-  const int64_t tiles = (a.n + p.rt - 1) / p.rt;
-  const int64_t grid = std::min<int64_t>(d.num_sms, tiles);
   // programmatic dependent launch: the kernel's first weight stages stream
   // while the stream's previous kernel drains (the kernel waits for it before
   // touching activations or outputs)

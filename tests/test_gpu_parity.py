@@ -177,8 +177,9 @@ def test_linear_within_tolerance_workloads(name):
 
 
 @pytest.mark.parametrize("path", ["gemv", "auto"])
+# (1, 300, 17408) and (2, 150, 8192): rows longer than a stage, streamed in chunks
 @pytest.mark.parametrize("m,n,k", [(1, 1000, 768), (3, 37, 2304), (13, 64, 512), (5, 9, 4352), (2, 333, 1280),
-                                   (8, 77, 1536)])
+                                   (8, 77, 1536), (1, 300, 17408), (2, 150, 8192)])
 def test_linear_within_tolerance_ragged(m, n, k, path):
     x, _, fmt, packed, W = case("decode", m=m, n=n, k=k, seed=11 + m + n + k)
     y64 = oracle_linear(x, fmt, packed)
@@ -281,7 +282,8 @@ def test_bounded_wait_reports_timeout_and_context_survives():
 
 @pytest.mark.parametrize("name,m,n,k", [("pr1", None, None, None), ("decode", None, None, None),
                                         ("verify8", None, None, None), ("decode", 3, 1000, 768),
-                                        ("decode", 5, 37, 2304), ("decode", 7, 40, 17408)])
+                                        ("decode", 5, 37, 2304), ("decode", 7, 40, 17408),
+                                        ("decode", 1, 300, 17408), ("decode", 2, 100, 8192)])
 def test_linear_bf16_fused_matches_two_call_path(name, m, n, k):
     """One-launch act + GEMV: codes and scales bit-exact against the oracle,
     y bit-identical to the two-call path and within tolerance of the oracle."""
@@ -297,7 +299,7 @@ def test_linear_bf16_fused_matches_two_call_path(name, m, n, k):
     # one launch (the GEMV with the quantiser fused) when m * k <= 16384, else
     # the activation kernel and iq8r_linear's own choice: the same arithmetic
     # as the two-call path through that kernel
-    fused = x.shape[0] * x.shape[1] <= 16384
+    fused = x.shape[0] <= 2 or x.shape[0] * x.shape[1] <= 16384
     y2 = gpu_linear(x, W, path=iq8r.IQ8R_PATH_GEMV if fused else iq8r.IQ8R_PATH_AUTO)
     assert np.array_equal(host_bits(y), y2)
     y64 = oracle_linear(x, fmt, packed)
