@@ -55,6 +55,8 @@ CONFIGS = {
     "verify16": (16, 17408, 5120, "g256", 2000),
     "verify128": (128, 17408, 5120, "g256", 500),
     "prefill": (8192, 5120, 17408, "g256", 20),
+    "decode_g128": (1, 5120, 17408, "g128", 20000),
+    "prefill_g128": (8192, 5120, 17408, "g128", 20),
     "lm_head1": (1, 5120, 151936, "g128", 2000),
     "lm_head8": (8, 5120, 151936, "g128", 1000),
 }
@@ -510,6 +512,88 @@ def run_ours(args, rank, world, local_rank):
     return out
 
 
+def run_rescore(args, rank, world, local_rank):
+    """Candidate rescoring (iq8r_rescore): args.rescore weight rows a token,
+    drawn at random over the whole weight, on the workload's weight and
+    tokens. One launch a step; the activation codes are computed once."""
+    import torch
+    import quantised_fwht128_act_b200 as iq8r
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    m, k, n, fmt, _ = CONFIGS[args.config]
+    m = getattr(args, "m", None) or m
+    C, K, W = args.rescore, args.steps, args.warmup
+    x0, (codes, sub, scale), wl = make_inputs(args.config, m)
+    weight = iq8r.IQ8RWeight.from_packed(codes, sub, scale, fmt, True, device=dev)
+    xd = torch.from_numpy(x0.view(np.int16)).to(dev).view(torch.bfloat16)
+    xq, xs = iq8r.iq8r_rotate_quant_act(xd, True)
+    R = 8
+    g = torch.Generator(device="cpu").manual_seed(77 + rank)
+    cands = [torch.randint(0, n, (m, C), generator=g, dtype=torch.int32).to(dev) for _ in range(R)]
+    outs = [torch.empty((m, C), dtype=torch.bfloat16, device=dev) for _ in range(R)]
+    stream = torch.cuda.Stream(device=dev)
+    with torch.cuda.stream(stream):
+        for j in range(W):
+            iq8r.iq8r_rescore(xq, xs, weight, cands[j % R], outs[j % R])
+    stream.synchronize()
+    iq8r.iq8r_get_device_error(stream)
+    try:
+        graph = torch.cuda.CUDAGraph(keep_graph=True)
+    except TypeError:
+        graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for j in range(K):
+            iq8r.iq8r_rescore(xq, xs, weight, cands[j % R], outs[j % R])
+    graph.instantiate()
+    with torch.cuda.stream(stream):
+        graph.replay()
+    stream.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t0w = time.time()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record()
+        graph.replay()
+        end.record()
+    stream.synchronize()
+    t1w = time.time()
+    sampler.stop()
+    iq8r.iq8r_get_device_error(stream)
+    ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    row = k + (k // 256 + 2 if fmt == "g256" else 2 * (k // 128))
+    step_b = m * C * row + m * k + 4 * m + 4 * m * C + 2 * m * C
+    hbm, _, peak_src = peaks()
+    avg = ms / K
+    value = job_value(step_b * K, world, ms) / 1e9
+    launches = graph_kernel_nodes(graph)
+    del graph
+    return {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K, "warmup": W,
+        "ms_per_step": avg, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "int8", "data": "synthetic",
+        "config": {"workload": f"{args.config} rescoring", "m": m, "k": k, "n": n, "format": fmt, "rotated": True,
+                   "candidates_per_token": C, "step": "iq8r_rescore (one launch)", "bytes_per_step": step_b,
+                   "l2": "candidate rows drawn at random over the whole weight", "parallelism": "single GPU"
+                   if world == 1 else f"replicas x{world}",
+                   "timing": "one CUDA graph of the K launches; events around the replay"},
+        "roofline": {"bound": "hbm", "kernel": "rescore_kernel", "achieved": value / world, "peak": hbm,
+                     "unit": "GB/s", "frac": value / world / hbm,
+                     "peak_source": f"{peak_src} HBM copy (MEASURED_PEAKS.json hbm_gbs)", "traffic": None,
+                     "algorithmic_bytes_per_launch": step_b, "avg_launch_ms": avg},
+        "clocks": sampler.summary(t0w, t1w),
+        "gpu_launches": None if launches is None else launches * 1,
+        "e2e": None,
+        "cpu_baseline": None,
+    }
+
+
 # ------------------------------------------------------------ CPU oracle
 
 def blas_threads():
@@ -597,6 +681,8 @@ def main(argv=None):
     ap.add_argument("--path", choices=["auto", "gemv", "tc"], default="auto",
                     help="force the linear's kernel (auto: the library's choice)")
     ap.add_argument("--m", type=int, default=None, help="override the workload's token count M")
+    ap.add_argument("--rescore", type=int, default=0,
+                    help="time candidate rescoring (this many weight rows a token) instead of the layer")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the prefill TOPS line of the decode run")
@@ -625,6 +711,11 @@ def main(argv=None):
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
+        if args.rescore:
+            out = run_rescore(args, rank, world, local_rank)
+            if rank == 0:
+                print(json.dumps(out), flush=True)
+            return 0
         out = run_ours(args, rank, world, local_rank)
         if args.config == "decode" and not args.no_prefill:
             # the metric's second half: prefill int8 TOPS on the tensor cores

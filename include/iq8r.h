@@ -189,6 +189,22 @@ iq8r_status iq8r_linear_ex(const int8_t* xq, const float* x_scale, int64_t m, co
 iq8r_status iq8r_linear_noalloc(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,
                                 uint16_t* y_bf16, cudaStream_t stream);
 
+/* Candidate rescoring: the linear's outputs for a short list of weight rows
+ * per token, out[t][j] = y[t][cand[t][j]] with y as iq8r_linear defines it
+ * (same block sums, same epilogue). The IQ8R page, row "Speculator": the
+ * drafter's 2-bit head proposes 32 candidates per position, which the engine
+ * rescores against the model's own int8 head.
+ *   xq, x_scale  as for iq8r_linear (xq 16-byte aligned)
+ *   w            any IQ8R weight (the lm_head: G128); k <= 49152
+ *   cand         device int32 [m][n_cand], row indices in [0, w->n)
+ *   out_bf16     device bf16 [m][n_cand] (out)
+ * One launch, one warp per candidate. Trunk-format results are the same bits
+ * as the GEMV path of iq8r_linear. A candidate outside [0, n) gets output 0
+ * and makes the next iq8r_get_device_error return IQ8R_ERR_INVALID_ARG; no
+ * out-of-range row is read. */
+iq8r_status iq8r_rescore(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,
+                         const int32_t* cand, int64_t n_cand, uint16_t* out_bf16, cudaStream_t stream);
+
 /* Debug twin of iq8r_linear: writes the exact per-block int32 partial sums
  * P[i][j][g] = sum_{k in block g} xq[i][k] * codes[n0 + j][k] for rows
  * n0 <= n < n1 instead of y, computed by the same kernel code as the
@@ -200,7 +216,8 @@ iq8r_status iq8r_linear_partials(const int8_t* xq, int64_t m, const iq8r_weight*
 /* Synchronises `stream`, then reads and clears the current device's error
  * word. IQ8R_OK if no kernel reported a problem since the last call;
  * IQ8R_ERR_DEVICE_TIMEOUT if a bounded wait ran out (the message names the
- * kernel and the wait); IQ8R_ERR_CUDA if the stream itself failed. */
+ * kernel and the wait); IQ8R_ERR_INVALID_ARG if iq8r_rescore met a candidate
+ * index out of range; IQ8R_ERR_CUDA if the stream itself failed. */
 iq8r_status iq8r_get_device_error(cudaStream_t stream);
 
 /* Failure-path self-test (no counterpart on the pages). Launches one

@@ -83,6 +83,12 @@ WORKLOADS: dict[str, Workload] = {
     "verify16": Workload("verify16", m=16, k=17408, n=5120, fmt="g256", seed=2, w_outlier_frac=0.01, x_outliers=8),
     "verify128": Workload("verify128", m=128, k=17408, n=5120, fmt="g256", seed=2, w_outlier_frac=0.01, x_outliers=8),
     "prefill": Workload("prefill", m=8192, k=5120, n=17408, fmt="g256", seed=3, w_outlier_frac=0.01, x_outliers=8),
+    # the trunk in the earlier IQ8R format: a bf16 scale per (row, 128 of K)
+    # instead of u8 under a bf16 row scale (IQ8R page, introduction)
+    "decode_g128": Workload("decode_g128", m=1, k=5120, n=17408, fmt="g128", seed=1, w_outlier_frac=0.01,
+                            x_outliers=8),
+    "prefill_g128": Workload("prefill_g128", m=8192, k=5120, n=17408, fmt="g128", seed=3, w_outlier_frac=0.01,
+                             x_outliers=8),
     "lm_head1": Workload("lm_head1", m=1, k=5120, n=151936, fmt="g128", seed=4, w_outlier_frac=0.0, x_outliers=8),
     "lm_head8": Workload("lm_head8", m=8, k=5120, n=151936, fmt="g128", seed=4, w_outlier_frac=0.0, x_outliers=8),
 }

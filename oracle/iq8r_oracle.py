@@ -61,6 +61,7 @@ __all__ = [
     "partials",
     "linear",
     "linear_bf16",
+    "rescore",
 ]
 
 GROUP_TRUNK = 256  # "a u8 scale per row and 256 of K" (IQ8R page, "Weights")
@@ -326,6 +327,41 @@ def linear(xq: np.ndarray, a: np.ndarray, fmt: str, codes: np.ndarray,
     if rotated:
         y = y / 128.0
     return y
+
+
+def rescore(xq: np.ndarray, a: np.ndarray, fmt: str, codes: np.ndarray, sub: np.ndarray | None,
+            scale_bits: np.ndarray, cand: np.ndarray, rotated: bool = True) -> np.ndarray:
+    """Candidate rescoring in float64, out64 [M, C]: the layer output of each
+    token at its C candidate weight rows, out[t, j] = y[t, cand[t, j]].
+
+    "Qwen3.8-27B IQ8R + DFlash2 -- radiance container", row "Speculator": the
+    drafter's 2-bit head proposes 32 candidates that are rescored against
+    the model's own head. Written per (token, candidate) pair with its own
+    int64 dot products (not a gather from ``linear``), so that the tests can
+    pin one against the other.
+    """
+    xq = np.asarray(xq, dtype=np.int64)
+    cand = np.asarray(cand, dtype=np.int64)
+    m, c = cand.shape
+    k = xq.shape[1]
+    g = GROUP_TRUNK if fmt == "g256" else GROUP_HEAD
+    ng = k // g
+    out = np.zeros((m, c), np.float64)
+    for t in range(m):
+        a64 = float(np.float32(a[t]))
+        for j in range(c):
+            r = int(cand[t, j])
+            w = np.asarray(codes[r], dtype=np.int64)
+            # P over each block of the row: exact integer dot products
+            P = (xq[t].reshape(ng, g) * w.reshape(ng, g)).sum(axis=1)
+            if fmt == "g256":
+                S = int((P * np.asarray(sub[r], dtype=np.int64)).sum())
+                v = a64 * float(bf16_to_f32(np.asarray([scale_bits[r]]))[0]) * float(S)
+            else:
+                s = bf16_to_f32(np.asarray(scale_bits[r])).astype(np.float64)
+                v = a64 * float((P.astype(np.float64) * s).sum())
+            out[t, j] = v / 128.0 if rotated else v
+    return out
 
 
 def linear_bf16(y64: np.ndarray) -> np.ndarray:

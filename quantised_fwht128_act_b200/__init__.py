@@ -24,7 +24,7 @@ __all__ = [
     "IQ8R_FMT_G256_U8_BF16", "IQ8R_FMT_G128_BF16", "IQ8R_PATH_AUTO", "IQ8R_PATH_GEMV", "IQ8R_PATH_TC",
     "IQ8RError", "IQ8RWeight", "lib", "lib_path",
     "iq8r_version", "iq8r_last_error", "iq8r_packed_sizes", "iq8r_pack", "iq8r_rotate_quant_act",
-    "iq8r_linear", "iq8r_linear_bf16", "iq8r_linear_ex", "iq8r_linear_noalloc", "iq8r_linear_partials",
+    "iq8r_linear", "iq8r_linear_bf16", "iq8r_linear_ex", "iq8r_linear_noalloc", "iq8r_linear_partials", "iq8r_rescore",
     "iq8r_get_device_error",
     "iq8r_selftest_wait_timeout",
 ]
@@ -94,6 +94,8 @@ def lib():
     L.iq8r_linear.argtypes = [vp, vp, i64, ctypes.POINTER(_Weight), vp, vp]
     L.iq8r_linear_bf16.restype = i32
     L.iq8r_linear_bf16.argtypes = [vp, i64, ctypes.POINTER(_Weight), vp, vp, vp, vp]
+    L.iq8r_rescore.restype = i32
+    L.iq8r_rescore.argtypes = [vp, vp, i64, ctypes.POINTER(_Weight), vp, i64, vp, vp]
     L.iq8r_linear_noalloc.restype = i32
     L.iq8r_linear_noalloc.argtypes = [vp, vp, i64, ctypes.POINTER(_Weight), vp, vp]
     L.iq8r_linear_ex.restype = i32
@@ -227,6 +229,18 @@ def iq8r_linear_ex(xq, x_scale, weight: IQ8RWeight, y=None, path: int = IQ8R_PAT
     w = weight._struct()
     _check(lib().iq8r_linear_ex(_ptr(xq), _ptr(x_scale), m, ctypes.byref(w), _ptr(y), path, _stream(stream)))
     return y
+
+
+def iq8r_rescore(xq, x_scale, weight: IQ8RWeight, cand, out=None, stream=None):
+    """out[t][j] = y[t][cand[t][j]] (int32 candidate rows [M, C]; bf16 [M, C])."""
+    import torch
+    m, c = cand.shape
+    if out is None:
+        out = torch.empty((m, c), dtype=torch.bfloat16, device=xq.device)
+    w = weight._struct()
+    _check(lib().iq8r_rescore(_ptr(xq), _ptr(x_scale), m, ctypes.byref(w), _ptr(cand), c, _ptr(out),
+                              _stream(stream)))
+    return out
 
 
 def iq8r_linear_noalloc(xq, x_scale, weight: IQ8RWeight, y=None, stream=None):

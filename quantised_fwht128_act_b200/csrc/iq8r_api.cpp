@@ -257,6 +257,24 @@ iq8r_status iq8r_linear_partials(const int8_t* xq, int64_t m, const iq8r_weight*
   return run_linear(a, path, fn, stream);
 }
 
+iq8r_status iq8r_rescore(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,
+                         const int32_t* cand, int64_t n_cand, uint16_t* out_bf16, cudaStream_t stream) {
+  const char* fn = "iq8r_rescore";
+  iq8r_status st = check_weight(w, fn);
+  if (st != IQ8R_OK) return st;
+  if (m < 0 || m > kMaxGridRows) return fail(IQ8R_ERR_INVALID_ARG, "%s: m = %lld out of range", fn, (long long)m);
+  if (n_cand < 0 || n_cand > 65535 * 32)
+    return fail(IQ8R_ERR_INVALID_ARG, "%s: n_cand = %lld out of range", fn, (long long)n_cand);
+  if (w->k > 48 * 1024) return fail(IQ8R_ERR_UNSUPPORTED, "%s: k above 49152 is not supported", fn);
+  if (m == 0 || n_cand == 0) return ok();
+  if (!xq || !x_scale || !cand || !out_bf16) return fail(IQ8R_ERR_INVALID_ARG, "%s: NULL buffer", fn);
+  if (!aligned16(xq)) return fail(IQ8R_ERR_INVALID_ARG, "%s: xq must be 16-byte aligned", fn);
+  iq8r::LinearArgs a = make_args(xq, x_scale, m, w);
+  const cudaError_t e = iq8r::launch_rescore(a, cand, static_cast<int>(n_cand), out_bf16, stream);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
+}
+
 iq8r_status iq8r_get_device_error(cudaStream_t stream) {
   cudaError_t e = cudaStreamSynchronize(stream);
   if (e != cudaSuccess) return cuda_fail(e, "iq8r_get_device_error: stream");
@@ -275,6 +293,8 @@ iq8r_status iq8r_get_device_error(cudaStream_t stream) {
     case iq8r::kDevErrTcAccEmpty: what = "TC GEMM MMA waiting for a drained accumulator"; break;
     case iq8r::kDevErrTcDrain: what = "TC GEMM draining its copies"; break;
     case iq8r::kDevErrSelftest: what = "self-test wait (expected)"; break;
+    case iq8r::kDevErrRescoreIndex:
+      return fail(IQ8R_ERR_INVALID_ARG, "iq8r_rescore: a candidate index was outside [0, n) (its output is 0)");
     default: break;
   }
   return fail(IQ8R_ERR_DEVICE_TIMEOUT, "device wait timed out: %s (code 0x%x)", what, code);

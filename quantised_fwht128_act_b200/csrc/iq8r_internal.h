@@ -26,6 +26,7 @@ enum DeviceError : uint32_t {
   kDevErrTcAccEmpty = 0x204,  // TC GEMM: accumulator never drained
   kDevErrTcDrain = 0x205,     // TC GEMM: copy in flight at exit
   kDevErrSelftest = 0x301,    // self-test wait that nothing satisfies
+  kDevErrRescoreIndex = 0x401,  // rescoring: a candidate row index outside [0, n)
 };
 
 struct LinearArgs {
@@ -59,6 +60,8 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_
 bool gemm_tc_supported(const LinearArgs& a, std::string* why);
 cudaError_t read_and_clear_device_error(uint32_t* err);
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
+// out[t][j] = y[t][cand[t][j]] (see rescore.cuh)
+cudaError_t launch_rescore(const LinearArgs& a, const int32_t* cand, int kc, uint16_t* out, cudaStream_t stream);
 
 // Host packer (iq8r_pack.cpp).
 void pack_rows(int fmt, bool rotate, const uint16_t* w, int64_t n, int64_t k, int8_t* codes,

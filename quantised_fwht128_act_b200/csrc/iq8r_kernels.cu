@@ -11,6 +11,7 @@
 #include "act_quant.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "rescore.cuh"
 #include "iq8r_device.cuh"
 #include "iq8r_internal.h"
 
@@ -519,6 +520,37 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_
                 : launch_tc_t<0, false, kTcMaxBM>(tw, tx, p, grid, stream);
   return part ? launch_tc_t<1, true, kTcMaxBM>(tw, tx, p, grid, stream)
               : launch_tc_t<1, false, kTcMaxBM>(tw, tx, p, grid, stream);
+}
+
+cudaError_t launch_rescore(const LinearArgs& a, const int32_t* cand, int kc, uint16_t* out, cudaStream_t stream) {
+  if (a.m == 0 || kc == 0) return cudaSuccess;
+  RescoreArgs r{};
+  r.xq = a.xq;
+  r.xs = a.xs;
+  r.m = a.m;
+  r.codes = a.codes;
+  r.sub = a.sub;
+  r.scale = a.scale;
+  r.n = a.n;
+  r.k = static_cast<int>(a.k);
+  r.rotated = a.rotated;
+  r.cand = cand;
+  r.kc = kc;
+  r.out = out;
+  const dim3 grid(static_cast<unsigned>(a.m), static_cast<unsigned>((kc + kRescoreWarps - 1) / kRescoreWarps));
+  const size_t smem = static_cast<size_t>(a.k);
+  if (a.fmt == 0) {
+    static std::atomic<int> configured[kMaxDevices];
+    cudaError_t e = ensure_smem(rescore_kernel<0>, static_cast<int>(smem), configured);
+    if (e != cudaSuccess) return e;
+    rescore_kernel<0><<<grid, kRescoreWarps * 32, smem, stream>>>(r);
+  } else {
+    static std::atomic<int> configured[kMaxDevices];
+    cudaError_t e = ensure_smem(rescore_kernel<1>, static_cast<int>(smem), configured);
+    if (e != cudaSuccess) return e;
+    rescore_kernel<1><<<grid, kRescoreWarps * 32, smem, stream>>>(r);
+  }
+  return cudaGetLastError();
 }
 
 namespace {

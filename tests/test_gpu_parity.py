@@ -12,7 +12,7 @@ import torch
 
 import oracle
 import quantised_fwht128_act_b200 as iq8r
-from iq8r_inputs import f32_to_bf16_bits, gen_workload
+from iq8r_inputs import WORKLOADS, f32_to_bf16_bits, gen_workload
 from tolerance import check_output
 
 pytestmark = pytest.mark.gpu
@@ -39,7 +39,7 @@ def built():
 def case(name, m=None, n=None, k=None, seed=None):
     """Inputs, oracle-packed weight and device copies for one configuration."""
     x, w = gen_workload(name, m=m, n=n, k=k, seed=seed)
-    fmt = "g128" if name.startswith("lm_head") else "g256"
+    fmt = WORKLOADS[name].fmt
     codes, sub, scale = oracle.pack(w, fmt, True)
     W = iq8r.IQ8RWeight.from_packed(codes, sub, scale, fmt, True)
     return x, w, fmt, (codes, sub, scale), W
@@ -365,6 +365,21 @@ def test_tc_lm_head_format():
     check_output(gpu_linear(x, W, path=iq8r.IQ8R_PATH_TC), y64, oracle.linear_bf16(y64))
 
 
+# the trunk in the earlier IQ8R format (a bf16 scale per row and 128 of K):
+# the lm_head kernels at trunk shapes, through both kernels
+@pytest.mark.parametrize("path", ["gemv", "tc"])
+@pytest.mark.parametrize("m,n,k", [(1, 17408, 5120), (16, 512, 17408), (300, 640, 5120)])
+def test_trunk_g128_format(m, n, k, path):
+    x, _, fmt, packed, W = case("decode_g128", m=m, n=n, k=k, seed=61 + m)
+    assert fmt == "g128"
+    p = iq8r.IQ8R_PATH_GEMV if path == "gemv" else iq8r.IQ8R_PATH_TC
+    xq, _ = oracle.act_quant(x)
+    rows = slice(0, min(n, 2048))
+    assert np.array_equal(gpu_partials(x, W, 0, rows.stop, path=p), oracle.partials(xq, packed[0][rows], 128))
+    y64 = oracle_linear(x, fmt, packed)
+    check_output(gpu_linear(x, W, path=p), y64, oracle.linear_bf16(y64))
+
+
 # few output tiles and long K: the tile's K range is split over several CTAs
 # and the fp32 partial tiles are added by the tile's last unit
 TC_SPLIT_SHAPES = [(16, 256, 17408), (128, 384, 8192), (8, 200, 4096), (40, 130, 2560), (96, 1, 1024)]
@@ -399,3 +414,50 @@ def test_tc_and_gemv_agree_on_partials():
     a = gpu_partials(x, W, path=iq8r.IQ8R_PATH_TC)
     b = gpu_partials(x, W, path=iq8r.IQ8R_PATH_GEMV)
     assert np.array_equal(a, b)
+
+
+# ------------------------------------------------------------- rescoring
+
+def _rescore_case(name, m, n, k, seed, n_cand=32):
+    x, _, fmt, packed, W = case(name, m=m, n=n, k=k, seed=seed)
+    rng = np.random.default_rng(seed)
+    cand = rng.integers(0, n, size=(m, n_cand)).astype(np.int32)
+    cand[0, :3] = [0, n - 1, 0]  # first and last rows, a duplicate
+    return x, fmt, packed, W, cand
+
+
+@pytest.mark.parametrize("name,m,n,k", [("lm_head8", 8, 4096, 5120), ("decode", 5, 2000, 5120),
+                                        ("decode_g128", 3, 1000, 2560), ("decode", 2, 300, 17408)])
+def test_rescore_matches_oracle_and_gemv(name, m, n, k):
+    """Candidate rescoring: within tolerance of the oracle, and the same bits
+    as the GEMV path of the full linear at the candidate rows."""
+    x, fmt, packed, W, cand = _rescore_case(name, m, n, k, seed=51 + m)
+    xq, xs = iq8r.iq8r_rotate_quant_act(dev_bf16(x))
+    cd = torch.from_numpy(cand).cuda()
+    got = host_bits(iq8r.iq8r_rescore(xq, xs, W, cd))
+    q, a = oracle.act_quant(x)
+    ref64 = oracle.rescore(q, a, fmt, *packed, cand)
+    check_output(got, ref64, oracle.linear_bf16(ref64))
+    full = host_bits(iq8r.iq8r_linear_ex(xq, xs, W, path=iq8r.IQ8R_PATH_GEMV))
+    assert np.array_equal(got, np.take_along_axis(full, cand.astype(np.int64), axis=1))
+    iq8r.iq8r_get_device_error()
+
+
+def test_rescore_out_of_range_candidate_is_reported():
+    x, fmt, packed, W, cand = _rescore_case("lm_head8", 2, 256, 1024, seed=57, n_cand=8)
+    cand[1, 4] = 256   # one past the last row
+    cand[0, 7] = -1
+    xq, xs = iq8r.iq8r_rotate_quant_act(dev_bf16(x))
+    out = host_bits(iq8r.iq8r_rescore(xq, xs, W, torch.from_numpy(cand).cuda()))
+    with pytest.raises(iq8r.IQ8RError) as err:
+        iq8r.iq8r_get_device_error()
+    assert err.value.status == iq8r.IQ8R_ERR_INVALID_ARG
+    assert out[1, 4] == 0 and out[0, 7] == 0
+    q, a = oracle.act_quant(x)
+    ok = cand.copy()
+    ok[1, 4] = ok[0, 7] = 0
+    ref = oracle.linear_bf16(oracle.rescore(q, a, fmt, *packed, ok))
+    mask = np.ones_like(cand, bool)
+    mask[1, 4] = mask[0, 7] = False
+    check_output(out[mask][None], oracle.rescore(q, a, fmt, *packed, ok)[mask][None], ref[mask][None])
+    iq8r.iq8r_get_device_error()  # the word was cleared by the read above

@@ -165,3 +165,22 @@ def test_workload_shapes_cover_the_pages_sizes():
     assert (WORKLOADS["decode"].k, WORKLOADS["decode"].n) == (5120, 17408)
     assert (WORKLOADS["verify128"].k, WORKLOADS["verify128"].n) == (17408, 5120)
     assert WORKLOADS["prefill"].m == 8192 and WORKLOADS["lm_head1"].n == 151936
+
+
+# ------------------------------------------------------------- rescoring
+
+@pytest.mark.parametrize("fmt", ["g256", "g128"])
+def test_rescore_is_the_linear_at_the_candidates(fmt):
+    """Rescoring (per pair, its own dot products) equals the full layer
+    output gathered at the candidate rows, duplicates and the first/last row
+    included; unrotated too."""
+    rng = np.random.default_rng(12)
+    x, w = gen_workload("decode", m=3, n=40, k=512, seed=12)
+    for rotated in (True, False):
+        codes, sub, scale = oracle.pack(w, fmt, rotated)
+        xq, a = oracle.act_quant(x, rotated)
+        y = oracle.linear(xq, a, fmt, codes, sub, scale, rotated=rotated)
+        cand = rng.integers(0, 40, size=(3, 6))
+        cand[0, :3] = [0, 39, 0]
+        got = oracle.rescore(xq, a, fmt, codes, sub, scale, cand, rotated=rotated)
+        assert np.array_equal(got, np.take_along_axis(y, cand, axis=1))
