@@ -113,6 +113,21 @@ iq8r_status iq8r_packed_sizes(int32_t fmt, int64_t n, int64_t k, size_t* codes_b
 iq8r_status iq8r_pack(int32_t fmt, int32_t rotate, const uint16_t* w_bf16, int64_t n, int64_t k,
                       int8_t* codes, uint8_t* sub_scale, uint16_t* scale, int32_t n_threads);
 
+/* Packing rules: IQ8R_RULE_RTN is iq8r_pack's. IQ8R_RULE_SEARCH is the
+ * recipes' "rule=search" ("a scale per 128 columns searched for least
+ * error", "Qwen3.8-Flash-Next, IQR-V4 -- radiance container", row "Trunk"),
+ * in this reading: per group, the RTN scale (the smallest that clips
+ * nothing) and the 15 next smaller ones are tried, and the one with the least
+ * sum of (w' - code * step)^2 over the group (in double, added in order)
+ * is kept, ties going to the larger scale. For the trunk the candidates are
+ * s1, s1 - 1, ... (>= 1) under the unchanged row scale s2; for G128 they are
+ * s and the next smaller bf16 values. */
+typedef enum { IQ8R_RULE_RTN = 0, IQ8R_RULE_SEARCH = 1 } iq8r_rule;
+
+/* iq8r_pack with a packing rule (same arguments otherwise). */
+iq8r_status iq8r_pack_ex(int32_t fmt, int32_t rotate, int32_t rule, const uint16_t* w_bf16, int64_t n,
+                         int64_t k, int8_t* codes, uint8_t* sub_scale, uint16_t* scale, int32_t n_threads);
+
 /* Rotate and quantise activations: "int8 under the same rotation (W8A8)"
  * (IQ8R page, "Activations"), one fp32 scale per token.
  *   x_bf16  device bf16 [m][k], raw 16-bit patterns, 16-byte aligned

@@ -57,6 +57,8 @@ __all__ = [
     "fwht128_f64",
     "act_quant",
     "pack",
+    "pack_search",
+    "SEARCH_WINDOW",
     "packed_sizes",
     "partials",
     "linear",
@@ -276,6 +278,96 @@ def pack(w_bits: np.ndarray, fmt: str = "g256", rotate: bool = True):
             t = blocks[sz] / s[sz][:, None]
             codes[sz] = np.clip(np.rint(t), -CODE_MAX, CODE_MAX).astype(np.int8)
         return codes.reshape(n, k), None, f32_to_bf16_exact(s)
+    raise ValueError(fmt)
+
+
+SEARCH_WINDOW = 16  # scale candidates tried by pack_search: the RTN scale and the 15 below it
+
+
+def _group_sse(blocks: np.ndarray, d: np.ndarray) -> np.ndarray:
+    """Squared reconstruction error of each group, sum over k in order.
+
+    blocks: float32 [..., G] rotated weights; d: float32 [...] steps (> 0).
+    Codes are the packer's (float32 divide, rint, clamp to +-127); each error
+    term is (w' - code * d) squared in float64 and the terms are added left
+    to right (a cumulative sum), the order the C++ packer uses.
+    """
+    q = np.clip(np.rint(blocks / d[..., None]), -CODE_MAX, CODE_MAX)
+    e = blocks.astype(np.float64) - q.astype(np.float64) * d[..., None].astype(np.float64)
+    return np.cumsum(e * e, axis=-1)[..., -1]
+
+
+def pack_search(w_bits: np.ndarray, fmt: str = "g256", rotate: bool = True, window: int = SEARCH_WINDOW):
+    """The recipes' ``rule=search``: per group, the scale with least
+    reconstruction error. "Qwen3.8-Flash-Next, IQR-V4 -- radiance
+    container", row "Trunk": "a scale per 128 columns searched for least
+    error"; the IQ8R recipe lines carry ``rule=search``.
+
+    Stated reading: start from the RTN scale of ``pack`` (the smallest that
+    clips nothing) and try it and the ``window - 1`` next smaller ones --
+    trunk: s1, s1 - 1, ... (s1 >= 1) under the unchanged row scale s2;
+    lm_head: s and the next smaller bf16 values (> 0). Smaller steps clip the
+    group's largest values but refine the rest. The error of a candidate is
+    the sum of (w' - code * step)**2 over the group (``_group_sse``); the
+    least wins, ties go to the larger scale. Same returns as ``pack``.
+    """
+    codes, sub, scale = pack(w_bits, fmt, rotate)
+    w = bf16_to_f32(w_bits)
+    n, k = w.shape
+    wr = fwht128_f32(w) if rotate else w.copy()
+    if fmt == "g256":
+        ng = k // GROUP_TRUNK
+        s2 = bf16_to_f32(scale)
+        sub = sub.copy()
+        codes = codes.reshape(n, ng, GROUP_TRUNK).copy()
+        for r0 in range(0, n, 256):  # rows in chunks: the candidates' errors take memory
+            r1 = min(n, r0 + 256)
+            blocks = wr[r0:r1].reshape(r1 - r0, ng, GROUP_TRUNK)
+            s1_rtn = sub[r0:r1].astype(np.float32)
+            best = np.full((r1 - r0, ng), np.inf)
+            best_s1 = s1_rtn.copy()
+            for i in range(window):
+                s1 = s1_rtn - np.float32(i)
+                ok = (s1 >= 1) & (s2[r0:r1, None] > 0)
+                d = np.where(ok, s2[r0:r1, None] * s1, np.float32(1))
+                sse = _group_sse(blocks, d)
+                better = ok & (sse < best)
+                best = np.where(better, sse, best)
+                best_s1 = np.where(better, s1, best_s1)
+            sub[r0:r1] = best_s1.astype(np.uint8)
+            d = s2[r0:r1, None] * best_s1
+            dz = d > 0
+            q = np.zeros(blocks.shape, np.int8)
+            if np.any(dz):
+                q[dz] = np.clip(np.rint(blocks[dz] / d[dz][:, None]), -CODE_MAX, CODE_MAX).astype(np.int8)
+            codes[r0:r1] = q
+        return codes.reshape(n, k), sub, scale
+    if fmt == "g128":
+        ng = k // GROUP_HEAD
+        scale = scale.copy()
+        codes = codes.reshape(n, ng, GROUP_HEAD).copy()
+        for r0 in range(0, n, 256):
+            r1 = min(n, r0 + 256)
+            blocks = wr[r0:r1].reshape(r1 - r0, ng, GROUP_HEAD)
+            b_rtn = scale[r0:r1].astype(np.int64)
+            best = np.full((r1 - r0, ng), np.inf)
+            best_b = b_rtn.copy()
+            for i in range(window):
+                b = b_rtn - i
+                ok = (b_rtn > 0) & (b >= 1)  # positive bf16 bit patterns: one step down is the next smaller value
+                s = bf16_to_f32(np.where(ok, b, 0x3F80).astype(np.uint16))
+                sse = _group_sse(blocks, s)
+                better = ok & (sse < best)
+                best = np.where(better, sse, best)
+                best_b = np.where(better, b, best_b)
+            scale[r0:r1] = best_b.astype(np.uint16)
+            s = bf16_to_f32(scale[r0:r1])
+            sz = s > 0
+            q = np.zeros(blocks.shape, np.int8)
+            if np.any(sz):
+                q[sz] = np.clip(np.rint(blocks[sz] / s[sz][:, None]), -CODE_MAX, CODE_MAX).astype(np.int8)
+            codes[r0:r1] = q
+        return codes.reshape(n, k), None, scale
     raise ValueError(fmt)
 
 

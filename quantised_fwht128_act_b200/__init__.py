@@ -22,6 +22,7 @@ import numpy as np
 __all__ = [
     "IQ8R_OK", "IQ8R_ERR_INVALID_ARG", "IQ8R_ERR_UNSUPPORTED", "IQ8R_ERR_CUDA", "IQ8R_ERR_DEVICE_TIMEOUT",
     "IQ8R_FMT_G256_U8_BF16", "IQ8R_FMT_G128_BF16", "IQ8R_PATH_AUTO", "IQ8R_PATH_GEMV", "IQ8R_PATH_TC",
+    "IQ8R_RULE_RTN", "IQ8R_RULE_SEARCH",
     "IQ8RError", "IQ8RWeight", "lib", "lib_path",
     "iq8r_version", "iq8r_last_error", "iq8r_packed_sizes", "iq8r_pack", "iq8r_rotate_quant_act",
     "iq8r_linear", "iq8r_linear_bf16", "iq8r_linear_ex", "iq8r_linear_noalloc", "iq8r_linear_partials", "iq8r_rescore",
@@ -29,6 +30,8 @@ __all__ = [
     "iq8r_selftest_wait_timeout",
 ]
 
+IQ8R_RULE_RTN = 0
+IQ8R_RULE_SEARCH = 1
 IQ8R_OK = 0
 IQ8R_ERR_INVALID_ARG = 1
 IQ8R_ERR_UNSUPPORTED = 2
@@ -88,6 +91,8 @@ def lib():
     L.iq8r_packed_sizes.argtypes = [i32, i64, i64, ctypes.POINTER(sz), ctypes.POINTER(sz), ctypes.POINTER(sz)]
     L.iq8r_pack.restype = i32
     L.iq8r_pack.argtypes = [i32, i32, vp, i64, i64, vp, vp, vp, i32]
+    L.iq8r_pack_ex.restype = i32
+    L.iq8r_pack_ex.argtypes = [i32, i32, i32, vp, i64, i64, vp, vp, vp, i32]
     L.iq8r_rotate_quant_act.restype = i32
     L.iq8r_rotate_quant_act.argtypes = [vp, i64, i64, i32, vp, vp, vp]
     L.iq8r_linear.restype = i32
@@ -154,10 +159,12 @@ def iq8r_packed_sizes(fmt, n: int, k: int):
     return c.value, s.value, sc.value
 
 
-def iq8r_pack(w_bf16, fmt="g256", rotate: bool = True, n_threads: int = 0):
+def iq8r_pack(w_bf16, fmt="g256", rotate: bool = True, n_threads: int = 0, rule: str = "rtn"):
     """Pack a host bf16 weight [N, K] (numpy uint16 bit patterns, or a CPU
     torch tensor of bf16 / int16 / uint16). Returns numpy arrays
-    (codes int8 [N, K], sub uint8 [N, K/256] or None, scale uint16 bits)."""
+    (codes int8 [N, K], sub uint8 [N, K/256] or None, scale uint16 bits).
+    rule: "rtn" (round to nearest) or "search" (least-error scales, see
+    include/iq8r.h)."""
     f = _fmt(fmt)
     if not isinstance(w_bf16, np.ndarray):
         import torch
@@ -173,7 +180,9 @@ def iq8r_pack(w_bf16, fmt="g256", rotate: bool = True, n_threads: int = 0):
     else:
         sub = None
         scale = np.empty((n, k // 128), np.uint16)
-    _check(lib().iq8r_pack(f, int(bool(rotate)), _ptr(w), n, k, _ptr(codes), _ptr(sub), _ptr(scale), n_threads))
+    rl = {"rtn": IQ8R_RULE_RTN, "search": IQ8R_RULE_SEARCH}[rule]
+    _check(lib().iq8r_pack_ex(f, int(bool(rotate)), rl, _ptr(w), n, k, _ptr(codes), _ptr(sub), _ptr(scale),
+                              n_threads))
     return codes, sub, scale
 
 

@@ -147,7 +147,14 @@ iq8r_status iq8r_packed_sizes(int32_t fmt, int64_t n, int64_t k, size_t* codes_b
 
 iq8r_status iq8r_pack(int32_t fmt, int32_t rotate, const uint16_t* w_bf16, int64_t n, int64_t k, int8_t* codes,
                       uint8_t* sub_scale, uint16_t* scale, int32_t n_threads) {
+  return iq8r_pack_ex(fmt, rotate, IQ8R_RULE_RTN, w_bf16, n, k, codes, sub_scale, scale, n_threads);
+}
+
+iq8r_status iq8r_pack_ex(int32_t fmt, int32_t rotate, int32_t rule, const uint16_t* w_bf16, int64_t n, int64_t k,
+                         int8_t* codes, uint8_t* sub_scale, uint16_t* scale, int32_t n_threads) {
   const char* fn = "iq8r_pack";
+  if (rule != IQ8R_RULE_RTN && rule != IQ8R_RULE_SEARCH)
+    return fail(IQ8R_ERR_INVALID_ARG, "%s: unknown rule %d", fn, rule);
   if (fmt != IQ8R_FMT_G256_U8_BF16 && fmt != IQ8R_FMT_G128_BF16)
     return fail(IQ8R_ERR_INVALID_ARG, "%s: unknown format %d", fn, fmt);
   if (rotate != 0 && rotate != 1) return fail(IQ8R_ERR_INVALID_ARG, "%s: rotate must be 0 or 1", fn);
@@ -158,8 +165,8 @@ iq8r_status iq8r_pack(int32_t fmt, int32_t rotate, const uint16_t* w_bf16, int64
   if (!w_bf16 || !codes || !scale) return fail(IQ8R_ERR_INVALID_ARG, "%s: NULL buffer", fn);
   if (fmt == IQ8R_FMT_G256_U8_BF16 && !sub_scale)
     return fail(IQ8R_ERR_INVALID_ARG, "%s: the trunk format needs sub_scale", fn);
-  iq8r::pack_rows(fmt, rotate != 0, w_bf16, n, k, codes, fmt == IQ8R_FMT_G256_U8_BF16 ? sub_scale : nullptr, scale,
-                  n_threads);
+  iq8r::pack_rows(fmt, rotate != 0, rule, w_bf16, n, k, codes, fmt == IQ8R_FMT_G256_U8_BF16 ? sub_scale : nullptr,
+                  scale, n_threads);
   return ok();
 }
 

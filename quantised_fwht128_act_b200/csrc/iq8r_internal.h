@@ -64,7 +64,7 @@ cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
 cudaError_t launch_rescore(const LinearArgs& a, const int32_t* cand, int kc, uint16_t* out, cudaStream_t stream);
 
 // Host packer (iq8r_pack.cpp).
-void pack_rows(int fmt, bool rotate, const uint16_t* w, int64_t n, int64_t k, int8_t* codes,
+void pack_rows(int fmt, bool rotate, int rule, const uint16_t* w, int64_t n, int64_t k, int8_t* codes,
                uint8_t* sub, uint16_t* scale, int n_threads);
 
 }  // namespace iq8r

@@ -9,7 +9,8 @@
 // bf16 scale per (row, 128 of K).
 //
 // The pages fit the codes by GPTQ against calibration Hessians; packing here
-// is the recipes' "rtn" rule with these stated scale definitions:
+// is the recipes' "rtn" rule with these stated scale definitions (and, on
+// request, rule=search over the scales below them, see pack_range):
 //   trunk:   s2 = bf16 of R / (127 * 255) rounded up, R the row's absmax;
 //            s1 = min(255, ceil(A / (127 * s2))), A the 256-block's absmax;
 //            code = clamp(rint(w' / (s2 * s1)), -127, 127).
@@ -79,7 +80,24 @@ inline int8_t quantise(float w, float step) {
   return static_cast<int8_t>(q);
 }
 
-void pack_range(int fmt, bool rotate, const uint16_t* w, int64_t k, int64_t r0, int64_t r1,
+// Squared reconstruction error of one group at step `d`: (w' - code * d)^2
+// in double, added in index order.
+inline double group_sse(const float* v, int64_t len, float d) {
+  double sse = 0.0;
+  for (int64_t i = 0; i < len; ++i) {
+    const double e = static_cast<double>(v[i]) - static_cast<double>(quantise(v[i], d)) * static_cast<double>(d);
+    sse += e * e;
+  }
+  return sse;
+}
+
+// The recipes' rule=search ("a scale per 128 columns searched for least
+// error", "Qwen3.8-Flash-Next, IQR-V4 -- radiance container", row "Trunk"):
+// the RTN step and the kSearchWindow - 1 next smaller ones, least error wins,
+// ties to the larger step.
+constexpr int kSearchWindow = 16;
+
+void pack_range(int fmt, bool rotate, int rule, const uint16_t* w, int64_t k, int64_t r0, int64_t r1,
                 int8_t* codes, uint8_t* sub, uint16_t* scale) {
   std::vector<float> row(static_cast<size_t>(k));
   const int64_t g256 = k / kGroupTrunk;
@@ -106,6 +124,20 @@ void pack_range(int fmt, bool rotate, const uint16_t* w, int64_t k, int64_t r0, 
       for (int64_t g = 0; g < g256; ++g) {
         float s1 = 0.0f;
         if (s2 > 0.0f) s1 = std::min(255.0f, std::ceil(amax[g] / den));
+        if (rule == 1 && s2 > 0.0f && s1 >= 1.0f) {
+          const float* v = row.data() + g * kGroupTrunk;
+          double best = group_sse(v, kGroupTrunk, s2 * s1);
+          float best_s1 = s1;
+          for (int i = 1; i < kSearchWindow && s1 - static_cast<float>(i) >= 1.0f; ++i) {
+            const float c = s1 - static_cast<float>(i);
+            const double e = group_sse(v, kGroupTrunk, s2 * c);
+            if (e < best) {
+              best = e;
+              best_s1 = c;
+            }
+          }
+          s1 = best_s1;
+        }
         sub[r * g256 + g] = static_cast<uint8_t>(s1);
         const float d = s2 * s1;  // exact: 8-bit x 8-bit significands
         for (int64_t i = g * kGroupTrunk; i < (g + 1) * kGroupTrunk; ++i) out[i] = quantise(row[i], d);
@@ -114,7 +146,21 @@ void pack_range(int fmt, bool rotate, const uint16_t* w, int64_t k, int64_t r0, 
       for (int64_t g = 0; g < g128; ++g) {
         float A = 0.0f;
         for (int64_t i = g * kGroupHead; i < (g + 1) * kGroupHead; ++i) A = std::max(A, std::fabs(row[i]));
-        const uint16_t sb = bf16_round_up_bits(A / 127.0f);
+        uint16_t sb = bf16_round_up_bits(A / 127.0f);
+        if (rule == 1 && sb > 0) {
+          const float* v = row.data() + g * kGroupHead;
+          double best = group_sse(v, kGroupHead, bf16_to_float(sb));
+          uint16_t best_b = sb;
+          for (int i = 1; i < kSearchWindow && static_cast<int>(sb) - i >= 1; ++i) {
+            const uint16_t c = static_cast<uint16_t>(sb - i);  // the next smaller positive bf16
+            const double e = group_sse(v, kGroupHead, bf16_to_float(c));
+            if (e < best) {
+              best = e;
+              best_b = c;
+            }
+          }
+          sb = best_b;
+        }
         scale[r * g128 + g] = sb;
         const float s = bf16_to_float(sb);
         for (int64_t i = g * kGroupHead; i < (g + 1) * kGroupHead; ++i) out[i] = quantise(row[i], s);
@@ -125,14 +171,14 @@ void pack_range(int fmt, bool rotate, const uint16_t* w, int64_t k, int64_t r0, 
 
 }  // namespace
 
-void pack_rows(int fmt, bool rotate, const uint16_t* w, int64_t n, int64_t k, int8_t* codes,
+void pack_rows(int fmt, bool rotate, int rule, const uint16_t* w, int64_t n, int64_t k, int8_t* codes,
                uint8_t* sub, uint16_t* scale, int n_threads) {
   if (n_threads <= 0) n_threads = static_cast<int>(std::max(1u, std::thread::hardware_concurrency()));
   const int64_t per = std::max<int64_t>(64, (n + n_threads - 1) / n_threads);
   std::vector<std::thread> pool;
   for (int64_t r0 = 0; r0 < n; r0 += per) {
     const int64_t r1 = std::min(n, r0 + per);
-    pool.emplace_back(pack_range, fmt, rotate, w, k, r0, r1, codes, sub, scale);
+    pool.emplace_back(pack_range, fmt, rotate, rule, w, k, r0, r1, codes, sub, scale);
   }
   for (auto& t : pool) t.join();
 }

@@ -170,3 +170,30 @@ def test_last_error_is_cleared_by_a_good_call(L):
     assert iq8r.iq8r_last_error() != ""
     iq8r.iq8r_packed_sizes("g256", 4, 256)
     assert iq8r.iq8r_last_error() == ""
+
+
+@pytest.mark.parametrize("fmt", ["g256", "g128"])
+def test_pack_search_byte_identical_to_oracle(L, fmt):
+    """rule=search: the C++ packer's chosen scales and codes are the
+    oracle's, on the workload generator and on edge rows (zero, a spike,
+    a constant row, tiny values)."""
+    _, w = gen_workload("decode", m=1, n=120, k=1024, seed=21)
+    w = w.copy()
+    w[3] = 0
+    w[4] = 0
+    w[4, 5] = f32_to_bf16_bits(np.array([3.0], np.float32))[0]
+    w[5] = f32_to_bf16_bits(np.full(1024, 0.25, np.float32))
+    w[6] = f32_to_bf16_bits(np.full(1024, 1e-30, np.float32))
+    got = iq8r.iq8r_pack(w, fmt, True, rule="search")
+    want = oracle.pack_search(w, fmt, True)
+    for g, e in zip(got, want):
+        assert (g is None and e is None) or np.array_equal(g, e)
+
+
+def test_pack_rule_is_checked(L):
+    w = np.zeros((2, 256), np.uint16)
+    codes = np.empty((2, 256), np.int8)
+    sub = np.empty((2, 1), np.uint8)
+    scale = np.empty((2,), np.uint16)
+    st = L.iq8r_pack_ex(0, 1, 7, w.ctypes.data, 2, 256, codes.ctypes.data, sub.ctypes.data, scale.ctypes.data, 1)
+    assert st == iq8r.IQ8R_ERR_INVALID_ARG

@@ -461,3 +461,21 @@ def test_rescore_out_of_range_candidate_is_reported():
     mask[1, 4] = mask[0, 7] = False
     check_output(out[mask][None], oracle.rescore(q, a, fmt, *packed, ok)[mask][None], ref[mask][None])
     iq8r.iq8r_get_device_error()  # the word was cleared by the read above
+
+
+# ---------------------------------------------- weights packed by rule=search
+
+@pytest.mark.parametrize("fmt,m,n,k,path", [("g256", 1, 3000, 5120, "gemv"), ("g256", 64, 640, 2560, "tc"),
+                                            ("g128", 8, 1000, 5120, "tc"), ("g128", 2, 700, 1024, "gemv")])
+def test_search_packed_weights(fmt, m, n, k, path):
+    """The kernels take least-error-packed weights as they are: partial sums
+    exact and outputs within tolerance of the oracle on the same packing."""
+    x, w = gen_workload("decode", m=m, n=n, k=k, seed=71 + m)
+    codes, sub, scale = iq8r.iq8r_pack(w, fmt, True, rule="search")
+    W = iq8r.IQ8RWeight.from_packed(codes, sub, scale, fmt, True)
+    p = iq8r.IQ8R_PATH_GEMV if path == "gemv" else iq8r.IQ8R_PATH_TC
+    q, a = oracle.act_quant(x)
+    g = 256 if fmt == "g256" else 128
+    assert np.array_equal(gpu_partials(x, W, path=p), oracle.partials(q, codes, g))
+    y64 = oracle.linear(q, a, fmt, codes, sub, scale, rotated=True)
+    check_output(gpu_linear(x, W, path=p), y64, oracle.linear_bf16(y64))

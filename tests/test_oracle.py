@@ -184,3 +184,51 @@ def test_rescore_is_the_linear_at_the_candidates(fmt):
         cand[0, :3] = [0, 39, 0]
         got = oracle.rescore(xq, a, fmt, codes, sub, scale, cand, rotated=rotated)
         assert np.array_equal(got, np.take_along_axis(y, cand, axis=1))
+
+
+# ------------------------------------------------------- rule=search packing
+
+def _exact_sse(vals, step):
+    """Exact (rational) squared error of a group at a step, codes as packed."""
+    from fractions import Fraction
+    tot = Fraction(0)
+    st = Fraction(float(step))
+    for v in vals:
+        q = max(-127, min(127, int(np.rint(np.float32(v) / np.float32(step)))))
+        e = Fraction(float(v)) - q * st
+        tot += e * e
+    return tot
+
+
+@pytest.mark.parametrize("fmt", ["g256", "g128"])
+def test_pack_search_minimises_group_error(fmt):
+    """Brute force: for every group of a small weight, the searched scale has
+    the least exact squared error among the RTN scale and the 15 below it
+    (ties to the larger); it never does worse than RTN, does better on some
+    groups, and the codes are those of the chosen scale."""
+    _, w = gen_workload("decode", m=1, n=6, k=512, seed=33)
+    wr = oracle.fwht128_f32(oracle.bf16_to_f32(w))
+    c0, s0, sc0 = oracle.pack(w, fmt, True)
+    c1, s1, sc1 = oracle.pack_search(w, fmt, True)
+    g = 256 if fmt == "g256" else 128
+    improved = 0
+    for r in range(w.shape[0]):
+        for b in range(w.shape[1] // g):
+            vals = wr[r, b * g:(b + 1) * g]
+            if fmt == "g256":
+                s2 = float(oracle.bf16_to_f32(sc0[r:r + 1])[0])
+                cands = [np.float32(s2) * np.float32(s0[r, b] - i) for i in range(16) if s0[r, b] - i >= 1]
+                chosen = np.float32(s2) * np.float32(s1[r, b])
+            else:
+                base = int(sc0[r, b])
+                cands = [oracle.bf16_to_f32(np.array([base - i], np.uint16))[0] for i in range(16) if base - i >= 1]
+                chosen = oracle.bf16_to_f32(sc1[r:r + 1, b])[0]
+            errs = [_exact_sse(vals, c) for c in cands]
+            best = min(errs)
+            e_chosen = _exact_sse(vals, chosen)
+            assert float(e_chosen) <= float(best) * (1 + 1e-9)
+            assert e_chosen <= errs[0]
+            improved += e_chosen < errs[0]
+            q = np.clip(np.rint(vals / np.float32(chosen)), -127, 127).astype(np.int8)
+            assert np.array_equal(c1[r, b * g:(b + 1) * g], q)
+    assert improved > 0

@@ -132,3 +132,21 @@ def test_transposed_weight_blocks_are_caught():
         return c, s1, s2
 
     fails(lambda: pins.check_product_identity(oracle.act_quant, pack_swapped_halves, oracle.linear, X, W, "g256"))
+
+
+def test_search_picking_the_worst_scale_is_caught(monkeypatch):
+    """rule=search that keeps the largest error instead of the least."""
+    import test_oracle
+    real = om._group_sse
+    monkeypatch.setattr(om, "_group_sse", lambda blocks, d: -real(blocks, d))
+    with pytest.raises(AssertionError):
+        test_oracle.test_pack_search_minimises_group_error("g128")
+
+
+def test_search_with_a_misplaced_step_is_caught(monkeypatch):
+    """rule=search that scores candidates at one step and keeps another."""
+    import test_oracle
+    real = om._group_sse
+    monkeypatch.setattr(om, "_group_sse", lambda blocks, d: real(blocks, d * np.float32(1.01)))
+    with pytest.raises(AssertionError):
+        test_oracle.test_pack_search_minimises_group_error("g256")
