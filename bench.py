@@ -57,6 +57,9 @@ CONFIGS = {
     "prefill": (8192, 5120, 17408, "g256", 20),
     "decode_g128": (1, 5120, 17408, "g128", 20000),
     "prefill_g128": (8192, 5120, 17408, "g128", 20),
+    # the drafter's codebook format at the trunk's shape (the pages give no
+    # drafter sizes)
+    "draft_cb4": (1, 5120, 17408, "cb4", 20000),
     "lm_head1": (1, 5120, 151936, "g128", 2000),
     "lm_head8": (8, 5120, 151936, "g128", 1000),
 }
@@ -73,6 +76,8 @@ def linear_bytes(m, k, n, fmt):
     """Weights (codes + scales), int8 activations + scales in, bf16 out."""
     if fmt == "g256":
         w = n * k + n * (k // 256) + 2 * n
+    elif fmt == "cb4":
+        w = n * k // 2 + 2 * n * (k // 128)
     else:
         w = n * k + 2 * n * (k // 128)
     return w + m * k + 4 * m + 2 * m * n
@@ -89,7 +94,9 @@ def fused_bytes(m, k, n, fmt):
 FUSE_MAX_M, FUSE_MAX_ELEMS, GEMV_MAX_M = 8, 16384, 2
 
 
-def one_launch(m, k):
+def one_launch(m, k, fmt="g256"):
+    if fmt == "cb4":  # the codebook format has no fused quantiser: two launches
+        return False
     return m <= GEMV_MAX_M or (m <= FUSE_MAX_M and m * k <= FUSE_MAX_ELEMS)
 
 
@@ -97,7 +104,7 @@ def step_bytes(m, k, n, fmt, fused=None):
     """Algorithmic bytes of one step: the fused layer (one launch), else the
     activation kernel plus the linear."""
     if fused is None:
-        fused = one_launch(m, k)
+        fused = one_launch(m, k, fmt)
     if fused:
         return fused_bytes(m, k, n, fmt)
     return act_bytes(m, k) + linear_bytes(m, k, n, fmt)
@@ -147,7 +154,7 @@ def is_hbm_bound(m, k, n, fmt, fused=None):
     the tensor cores above it. Decode and verify steps are HBM-bound and are
     reported in GB/s; prefill is tensor-bound and reported in int8 TOPS."""
     if fused is None:
-        fused = one_launch(m, k)
+        fused = one_launch(m, k, fmt)
     hbm, bf16_tf, _ = peaks()
     lin_b = fused_bytes(m, k, n, fmt) if fused else linear_bytes(m, k, n, fmt)
     return 2.0 * m * n * k / lin_b < bf16_tf * INT8_OVER_BF16 * 1e12 / (hbm * 1e9)
@@ -297,7 +304,8 @@ def run_ours(args, rank, world, local_rank):
     xsc = [torch.empty((m,), dtype=torch.float32, device=dev) for _ in range(R)]
     y = [torch.empty((m, n), dtype=torch.bfloat16, device=dev) for _ in range(R)]
     path = {"auto": iq8r.IQ8R_PATH_AUTO, "gemv": iq8r.IQ8R_PATH_GEMV, "tc": iq8r.IQ8R_PATH_TC}[args.path]
-    fused = one_launch(m, k) and args.path == "auto"  # the GEMV rotates and quantises x itself
+    # the GEMV rotates and quantises x itself (not for the codebook format)
+    fused = one_launch(m, k, fmt) and args.path == "auto"
 
     def linear(r):
         iq8r.iq8r_linear_ex(xq[r], xsc[r], weights[r], y[r], path=path)
@@ -453,10 +461,13 @@ def run_ours(args, rank, world, local_rank):
     # which the tensor peak and the HBM peak take equal time), tensor above
     hbm_bound = is_hbm_bound(m, k, n, fmt, fused)
     on_tc = args.path == "tc" or (args.path == "auto" and not fused and m > GEMV_MAX_M)
-    kname = ("gemv_kernel (fused act, one launch per step)" if fused else
+    on_tc = on_tc and fmt != "cb4"  # the codebook format has its own GEMV only
+    kname = ("cb4_gemv_kernel" if fmt == "cb4" else
+             "gemv_kernel (fused act, one launch per step)" if fused else
              "gemm_tc_kernel (tcgen05 kind::i8)" if on_tc else "gemv_kernel")
-    kfiles = ["gemm_tc.cuh", "iq8r_device.cuh"] if on_tc else ["gemv.cuh", "act_quant.cuh", "iq8r_device.cuh"]
-    ktraffic = recorded_traffic("gemm_tc_kernel" if on_tc else "gemv_kernel", args.config, kfiles)
+    kfiles = (["cb4_gemv.cuh", "iq8r_device.cuh"] if fmt == "cb4" else
+              ["gemm_tc.cuh", "iq8r_device.cuh"] if on_tc else ["gemv.cuh", "act_quant.cuh", "iq8r_device.cuh"])
+    ktraffic = recorded_traffic(kname.split(" ")[0], args.config, kfiles)
     if hbm_bound:
         achieved = lin_b / (lin_avg_ms * 1e-3) / 1e9
         roof = {"bound": "hbm", "kernel": kname, "achieved": achieved,
@@ -621,7 +632,7 @@ def run_oracle(cfg_name, budget_s, steps=None):
     m_s = min(m, 64)
     n_probe = min(n, 256)
     x, w = gen_workload(wl, m=m_s, n=n_probe, k=k)
-    packed = oracle.pack(w, fmt, True)
+    packed = oracle.pack(w, fmt, True) if fmt != "cb4" else (oracle.pack_cb4(w, True)[0], None, oracle.pack_cb4(w, True)[1])
     t = time.perf_counter()
     q, a = oracle.act_quant(x)
     oracle.linear(q, a, fmt, *packed, rotated=True)
@@ -634,7 +645,7 @@ def run_oracle(cfg_name, budget_s, steps=None):
         n_s = int(min(n, max(8, budget_s / steps / max(per_row, 1e-9))))
         reps = steps
     x, w = gen_workload(wl, m=m_s, n=n_s, k=k)
-    packed = oracle.pack(w, fmt, True)
+    packed = oracle.pack(w, fmt, True) if fmt != "cb4" else (oracle.pack_cb4(w, True)[0], None, oracle.pack_cb4(w, True)[1])
     del w
     t = time.perf_counter()
     for _ in range(reps):
@@ -642,7 +653,7 @@ def run_oracle(cfg_name, budget_s, steps=None):
         oracle.linear(q, a, fmt, *packed, rotated=True)
     dt = time.perf_counter() - t
     if is_hbm_bound(m, k, n, fmt):
-        b = step_bytes(m_s, k, n_s, fmt, fused=one_launch(m, k))
+        b = step_bytes(m_s, k, n_s, fmt, fused=one_launch(m, k, fmt))
         value, unit, what = b * reps / dt / 1e9, "GB/s", "algorithmic bytes"
     else:
         value, unit, what = 2.0 * m_s * n_s * k * reps / dt / 1e12, "TOPS", "int8 ops (2 M N K)"

@@ -65,7 +65,15 @@ typedef enum {
   /* trunk: int8 codes, u8 sub-scale per (row, 256 of K), bf16 scale per row */
   IQ8R_FMT_G256_U8_BF16 = 0,
   /* lm_head: int8 codes, bf16 scale per (row, 128 of K) */
-  IQ8R_FMT_G128_BF16 = 1
+  IQ8R_FMT_G128_BF16 = 1,
+  /* the drafter's linears: 4-bit indices into the 16 levels
+   * -127 -97 -75 -58 -43 -30 -18 -6 6 18 30 43 58 75 97 127 (IQ8R page,
+   * "How this file was made", the dflash recipe lines), two a byte with the
+   * even K position in the low nibble, and a bf16 scale per (row, 128 of K);
+   * y as for G128 with the codes' levels. Packed by nearest level (ties to
+   * the larger) under s = bf16 of A / 127 rounded up. GEMV only (any M, 8
+   * tokens a launch); not for iq8r_rescore. */
+  IQ8R_FMT_CB4_G128 = 2
 } iq8r_format;
 
 /* Kernel choice for iq8r_linear_ex. AUTO picks by M. */
@@ -76,7 +84,8 @@ typedef enum {
 } iq8r_path;
 
 /* A packed weight on the device. Not owned by the library.
- *   codes     int8 [n][k], K contiguous (row-major), values -127..127
+ *   codes     int8 [n][k], K contiguous (row-major), values -127..127; for
+ *             IQ8R_FMT_CB4_G128 the packed indices, u8 [n][k/2]
  *   sub_scale u8   [n][k/256] for IQ8R_FMT_G256_U8_BF16; NULL for G128
  *   scale     bf16 [n] (G256) or [n][k/128] (G128), as raw 16-bit patterns
  *   rotated   1 if the codes live in the fwht128 domain (the output is then

@@ -63,7 +63,7 @@ class Workload:
     m: int
     k: int
     n: int
-    fmt: str  # "g256" (trunk: u8 per 256 under a bf16 row scale) or "g128" (bf16 per 128)
+    fmt: str  # "g256" (trunk: u8 per 256 under a bf16 row scale), "g128" (bf16 per 128), "cb4" (codebook)
     seed: int
     w_outlier_frac: float
     x_outliers: int
@@ -89,6 +89,8 @@ WORKLOADS: dict[str, Workload] = {
                             x_outliers=8),
     "prefill_g128": Workload("prefill_g128", m=8192, k=5120, n=17408, fmt="g128", seed=3, w_outlier_frac=0.01,
                              x_outliers=8),
+    # the drafter's linears in their codebook format, at the trunk's shape
+    "draft_cb4": Workload("draft_cb4", m=1, k=5120, n=17408, fmt="cb4", seed=5, w_outlier_frac=0.01, x_outliers=8),
     "lm_head1": Workload("lm_head1", m=1, k=5120, n=151936, fmt="g128", seed=4, w_outlier_frac=0.0, x_outliers=8),
     "lm_head8": Workload("lm_head8", m=8, k=5120, n=151936, fmt="g128", seed=4, w_outlier_frac=0.0, x_outliers=8),
 }

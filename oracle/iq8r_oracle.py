@@ -33,10 +33,17 @@ library follows it exactly):
 * rounding: round-half-to-even wherever a value is rounded to nearest;
 * the factor 1/128 (H H = 128 I) is applied to the output.
 
-Parity unpinned: the choice of the three scale rules above (per-token
-activation scale, the s2/s1 composition, the lm_head scale rule) and of the
-butterfly order. They are stated definitions, not facts the pages fix; the
-tests pin everything that follows from them.
+Also written here: ``pack_search`` (the recipes' rule=search: least-error
+scales among the RTN scale and the 15 below it), ``pack_cb4`` / ``decode_cb4``
+(the drafter's 16-level codebook: nearest level under s = bf16 of A / 127
+rounded up, ties to the larger level) and ``rescore`` (the layer at a list of
+candidate rows).
+
+Parity unpinned: the choice of the scale rules above (per-token activation
+scale, the s2/s1 composition, the lm_head scale rule, the search window and
+its error measure, the codebook's scale and tie rule) and of the butterfly
+order. They are stated definitions, not facts the pages fix; the tests pin
+everything that follows from them.
 """
 
 from __future__ import annotations
@@ -58,6 +65,9 @@ __all__ = [
     "act_quant",
     "pack",
     "pack_search",
+    "pack_cb4",
+    "decode_cb4",
+    "CB4_TABLE",
     "SEARCH_WINDOW",
     "packed_sizes",
     "partials",
@@ -71,6 +81,10 @@ GROUP_HEAD = 128   # "a bf16 scale per row and 128" (IQ8R page, "Weights")
 CODE_MAX = 127     # "codes -127..127", clamp=sym (IQ8R page, "Weights" and recipe)
 SUB_MAX = 255      # largest u8 sub-scale (recipe: scale=u8)
 ROT = 128          # fwht128: the rotation acts on each 128 of K
+# The drafter's 16-level integer codebook (IQ8R page, "How this file was
+# made": the dflash recipe lines, table=-127;-97;...;97;127, group=128
+# scale=bf16 transform=fwht128): index i (4 bits) stands for CB4_TABLE[i].
+CB4_TABLE = np.array([-127, -97, -75, -58, -43, -30, -18, -6, 6, 18, 30, 43, 58, 75, 97, 127], dtype=np.int64)
 
 
 # ---------------------------------------------------------------- bf16 helpers
@@ -217,6 +231,8 @@ def packed_sizes(fmt: str, n: int, k: int):
         return n * k, n * (k // GROUP_TRUNK), 2 * n
     if fmt == "g128":
         return n * k, 0, 2 * n * (k // GROUP_HEAD)
+    if fmt == "cb4":
+        return n * k // 2, 0, 2 * n * (k // GROUP_HEAD)
     raise ValueError(fmt)
 
 
@@ -279,6 +295,50 @@ def pack(w_bits: np.ndarray, fmt: str = "g256", rotate: bool = True):
             codes[sz] = np.clip(np.rint(t), -CODE_MAX, CODE_MAX).astype(np.int8)
         return codes.reshape(n, k), None, f32_to_bf16_exact(s)
     raise ValueError(fmt)
+
+
+def pack_cb4(w_bits: np.ndarray, rotate: bool = True):
+    """The drafter's codebook format: 4-bit indices into CB4_TABLE with a
+    bf16 scale per (row, 128 of K), in the rotated domain (the dflash recipe
+    lines: ``rtn table=... group=128 scale=bf16 transform=fwht128``).
+
+    Stated reading: s = bf16 of A / 127 rounded up (A the group's max |w'|,
+    so the end levels +-127 cover every value), and each value takes the
+    level nearest to w' / s (float32 divide), ties going to the larger level;
+    a group with s = 0 takes index 8 (level +6, contributing 0). Two indices a
+    byte, the even K position in the low nibble.
+
+    Returns (packed uint8 [N, K/2], scale bf16 bits [N, K/128]).
+    """
+    w = bf16_to_f32(w_bits)
+    n, k = w.shape
+    if k % GROUP_HEAD:
+        raise ValueError("K must be a multiple of 128")
+    wr = fwht128_f32(w) if rotate else w.copy()
+    ng = k // GROUP_HEAD
+    blocks = wr.reshape(n, ng, GROUP_HEAD)
+    A = np.max(np.abs(blocks), axis=2)
+    s = bf16_round_up(A / np.float32(CODE_MAX))
+    idx = np.full((n, ng, GROUP_HEAD), 8, dtype=np.uint8)
+    sz = s > 0
+    if np.any(sz):
+        t = (blocks[sz] / s[sz][:, None]).astype(np.float64)        # [groups, 128]
+        dist = np.abs(t[..., None] - CB4_TABLE.astype(np.float64))  # [groups, 128, 16]
+        # least distance, ties to the larger level: search from the top index down
+        rev = dist[..., ::-1]
+        idx[sz] = (15 - np.argmin(rev, axis=-1)).astype(np.uint8)
+    idx = idx.reshape(n, k)
+    packed = (idx[:, 0::2] | (idx[:, 1::2] << 4)).astype(np.uint8)
+    return packed, f32_to_bf16_exact(s)
+
+
+def decode_cb4(packed: np.ndarray) -> np.ndarray:
+    """The codebook values of packed indices: int8 [N, K]."""
+    p = np.asarray(packed, dtype=np.uint8)
+    idx = np.empty((p.shape[0], p.shape[1] * 2), dtype=np.uint8)
+    idx[:, 0::2] = p & 0x0F
+    idx[:, 1::2] = p >> 4
+    return CB4_TABLE[idx].astype(np.int8)
 
 
 SEARCH_WINDOW = 16  # scale candidates tried by pack_search: the RTN scale and the 15 below it
@@ -410,8 +470,10 @@ def linear(xq: np.ndarray, a: np.ndarray, fmt: str, codes: np.ndarray,
         S = np.einsum("mng,ng->mn", P, np.asarray(sub).astype(np.int64))
         s2 = bf16_to_f32(scale_bits).astype(np.float64)
         y = a64[:, None] * s2[None, :] * S.astype(np.float64)
-    elif fmt == "g128":
-        P = partials(xq, codes, GROUP_HEAD)
+    elif fmt in ("g128", "cb4"):
+        # cb4: codes are the packed indices; their values are the codebook's
+        vals = decode_cb4(codes) if fmt == "cb4" else codes
+        P = partials(xq, vals, GROUP_HEAD)
         s = bf16_to_f32(scale_bits).astype(np.float64)
         y = a64[:, None] * np.einsum("mng,ng->mn", P.astype(np.float64), s)
     else:

@@ -22,7 +22,7 @@ import numpy as np
 __all__ = [
     "IQ8R_OK", "IQ8R_ERR_INVALID_ARG", "IQ8R_ERR_UNSUPPORTED", "IQ8R_ERR_CUDA", "IQ8R_ERR_DEVICE_TIMEOUT",
     "IQ8R_FMT_G256_U8_BF16", "IQ8R_FMT_G128_BF16", "IQ8R_PATH_AUTO", "IQ8R_PATH_GEMV", "IQ8R_PATH_TC",
-    "IQ8R_RULE_RTN", "IQ8R_RULE_SEARCH",
+    "IQ8R_RULE_RTN", "IQ8R_RULE_SEARCH", "IQ8R_FMT_CB4_G128",
     "IQ8RError", "IQ8RWeight", "lib", "lib_path",
     "iq8r_version", "iq8r_last_error", "iq8r_packed_sizes", "iq8r_pack", "iq8r_rotate_quant_act",
     "iq8r_linear", "iq8r_linear_bf16", "iq8r_linear_ex", "iq8r_linear_noalloc", "iq8r_linear_partials", "iq8r_rescore",
@@ -40,12 +40,13 @@ IQ8R_ERR_DEVICE_TIMEOUT = 4
 
 IQ8R_FMT_G256_U8_BF16 = 0
 IQ8R_FMT_G128_BF16 = 1
+IQ8R_FMT_CB4_G128 = 2
 
 IQ8R_PATH_AUTO = 0
 IQ8R_PATH_GEMV = 1
 IQ8R_PATH_TC = 2
 
-_FMT_NAMES = {"g256": IQ8R_FMT_G256_U8_BF16, "g128": IQ8R_FMT_G128_BF16}
+_FMT_NAMES = {"g256": IQ8R_FMT_G256_U8_BF16, "g128": IQ8R_FMT_G128_BF16, "cb4": IQ8R_FMT_CB4_G128}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 lib_path = os.path.join(_HERE, "libiq8r.so")
@@ -162,7 +163,8 @@ def iq8r_packed_sizes(fmt, n: int, k: int):
 def iq8r_pack(w_bf16, fmt="g256", rotate: bool = True, n_threads: int = 0, rule: str = "rtn"):
     """Pack a host bf16 weight [N, K] (numpy uint16 bit patterns, or a CPU
     torch tensor of bf16 / int16 / uint16). Returns numpy arrays
-    (codes int8 [N, K], sub uint8 [N, K/256] or None, scale uint16 bits).
+    (codes int8 [N, K] -- uint8 [N, K/2] packed indices for "cb4" --,
+    sub uint8 [N, K/256] or None, scale uint16 bits).
     rule: "rtn" (round to nearest) or "search" (least-error scales, see
     include/iq8r.h)."""
     f = _fmt(fmt)
@@ -173,7 +175,7 @@ def iq8r_pack(w_bf16, fmt="g256", rotate: bool = True, n_threads: int = 0, rule:
     if w.ndim != 2:
         raise ValueError("w must be [N, K]")
     n, k = w.shape
-    codes = np.empty((n, k), np.int8)
+    codes = np.empty((n, k // 2), np.uint8) if f == IQ8R_FMT_CB4_G128 else np.empty((n, k), np.int8)
     if f == IQ8R_FMT_G256_U8_BF16:
         sub = np.empty((n, k // 256), np.uint8)
         scale = np.empty((n,), np.uint16)
@@ -209,7 +211,9 @@ class IQ8RWeight:
             return t.to(device).contiguous()
 
         c = dev(codes)
-        return cls(_fmt(fmt), int(bool(rotated)), c.shape[0], c.shape[1], c, dev(sub), dev(scale))
+        f = _fmt(fmt)
+        k = c.shape[1] * 2 if f == IQ8R_FMT_CB4_G128 else c.shape[1]  # two indices a byte
+        return cls(f, int(bool(rotated)), c.shape[0], k, c, dev(sub), dev(scale))
 
     def _struct(self) -> _Weight:
         return _Weight(self.fmt, self.rotated, self.n, self.k, _ptr(self.codes), _ptr(self.sub_scale),

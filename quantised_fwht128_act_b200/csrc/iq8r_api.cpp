@@ -44,7 +44,7 @@ constexpr int64_t kGemvMaxM = 2;
 
 iq8r_status check_weight(const iq8r_weight* w, const char* fn) {
   if (!w) return fail(IQ8R_ERR_INVALID_ARG, "%s: weight is NULL", fn);
-  if (w->fmt != IQ8R_FMT_G256_U8_BF16 && w->fmt != IQ8R_FMT_G128_BF16)
+  if (w->fmt != IQ8R_FMT_G256_U8_BF16 && w->fmt != IQ8R_FMT_G128_BF16 && w->fmt != IQ8R_FMT_CB4_G128)
     return fail(IQ8R_ERR_INVALID_ARG, "%s: unknown weight format %d", fn, w->fmt);
   if (w->rotated != 0 && w->rotated != 1)
     return fail(IQ8R_ERR_INVALID_ARG, "%s: rotated must be 0 or 1", fn);
@@ -83,6 +83,14 @@ iq8r_status run_linear(const iq8r::LinearArgs& a, int32_t path, const char* fn, 
     return fail(IQ8R_ERR_INVALID_ARG, "%s: unknown path %d", fn, path);
   if (a.m == 0) return ok();
   std::string why;
+  if (a.fmt == IQ8R_FMT_CB4_G128) {
+    // the codebook format has one kernel, the weight-streaming GEMV
+    if (path == IQ8R_PATH_TC) return fail(IQ8R_ERR_UNSUPPORTED, "%s: the codebook format runs on the GEMV only", fn);
+    if (!iq8r::cb4_supported(a.k, &why)) return fail(IQ8R_ERR_UNSUPPORTED, "%s: %s", fn, why.c_str());
+    const cudaError_t e = iq8r::launch_cb4(a, stream);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return ok();
+  }
   bool use_tc = false;
   if (path == IQ8R_PATH_TC) {
     if (!iq8r::gemm_tc_supported(a, &why)) return fail(IQ8R_ERR_UNSUPPORTED, "%s: %s", fn, why.c_str());
@@ -128,13 +136,14 @@ const char* iq8r_last_error(void) { return t_last_error.c_str(); }
 
 iq8r_status iq8r_packed_sizes(int32_t fmt, int64_t n, int64_t k, size_t* codes_bytes, size_t* sub_bytes,
                               size_t* scale_bytes) {
-  if (fmt != IQ8R_FMT_G256_U8_BF16 && fmt != IQ8R_FMT_G128_BF16)
+  if (fmt != IQ8R_FMT_G256_U8_BF16 && fmt != IQ8R_FMT_G128_BF16 && fmt != IQ8R_FMT_CB4_G128)
     return fail(IQ8R_ERR_INVALID_ARG, "iq8r_packed_sizes: unknown format %d", fmt);
   const int64_t g = fmt == IQ8R_FMT_G256_U8_BF16 ? iq8r::kGroupTrunk : iq8r::kGroupHead;
   if (n < 0 || k < 0 || k % g)
     return fail(IQ8R_ERR_INVALID_ARG, "iq8r_packed_sizes: need n >= 0 and k a non-negative multiple of %lld",
                 (long long)g);
-  if (codes_bytes) *codes_bytes = static_cast<size_t>(n) * static_cast<size_t>(k);
+  if (codes_bytes)
+    *codes_bytes = static_cast<size_t>(n) * static_cast<size_t>(fmt == IQ8R_FMT_CB4_G128 ? k / 2 : k);
   if (fmt == IQ8R_FMT_G256_U8_BF16) {
     if (sub_bytes) *sub_bytes = static_cast<size_t>(n) * static_cast<size_t>(k / iq8r::kGroupTrunk);
     if (scale_bytes) *scale_bytes = 2 * static_cast<size_t>(n);
@@ -155,8 +164,10 @@ iq8r_status iq8r_pack_ex(int32_t fmt, int32_t rotate, int32_t rule, const uint16
   const char* fn = "iq8r_pack";
   if (rule != IQ8R_RULE_RTN && rule != IQ8R_RULE_SEARCH)
     return fail(IQ8R_ERR_INVALID_ARG, "%s: unknown rule %d", fn, rule);
-  if (fmt != IQ8R_FMT_G256_U8_BF16 && fmt != IQ8R_FMT_G128_BF16)
+  if (fmt != IQ8R_FMT_G256_U8_BF16 && fmt != IQ8R_FMT_G128_BF16 && fmt != IQ8R_FMT_CB4_G128)
     return fail(IQ8R_ERR_INVALID_ARG, "%s: unknown format %d", fn, fmt);
+  if (fmt == IQ8R_FMT_CB4_G128 && rule != IQ8R_RULE_RTN)
+    return fail(IQ8R_ERR_UNSUPPORTED, "%s: the codebook format packs by nearest level only", fn);
   if (rotate != 0 && rotate != 1) return fail(IQ8R_ERR_INVALID_ARG, "%s: rotate must be 0 or 1", fn);
   const int64_t g = fmt == IQ8R_FMT_G256_U8_BF16 ? iq8r::kGroupTrunk : iq8r::kGroupHead;
   if (n < 0 || k <= 0 || k % g)
@@ -211,7 +222,8 @@ iq8r_status iq8r_linear_bf16(const uint16_t* x_bf16, int64_t m, const iq8r_weigh
   // its rotation is cheap, or when there is nowhere to stage the codes.
   const bool small = m * w->k <= kFuseMaxElems;
   const bool staged = xq_out && x_scale_out;
-  if (m <= 8 && (small || m <= kGemvMaxM || !staged) && iq8r::gemv_supported(w->k, &why)) {
+  if (w->fmt != IQ8R_FMT_CB4_G128 && m <= 8 && (small || m <= kGemvMaxM || !staged) &&
+      iq8r::gemv_supported(w->k, &why)) {
     // one launch: every CTA rotates and quantises x itself, then streams W
     iq8r::LinearArgs a = make_args(nullptr, nullptr, m, w);
     a.y = y_bf16;
@@ -223,7 +235,7 @@ iq8r_status iq8r_linear_bf16(const uint16_t* x_bf16, int64_t m, const iq8r_weigh
     return ok();
   }
   if (!staged)
-    return fail(IQ8R_ERR_INVALID_ARG, "%s: m > 8 needs xq_out and x_scale_out (the codes are staged there)", fn);
+    return fail(IQ8R_ERR_INVALID_ARG, "%s: this call needs xq_out and x_scale_out (the codes are staged there)", fn);
   cudaError_t e = iq8r::launch_act_quant(x_bf16, m, w->k, w->rotated, xq_out, x_scale_out, stream);
   if (e != cudaSuccess) return cuda_fail(e, fn);
   iq8r::LinearArgs a = make_args(xq_out, x_scale_out, m, w);
@@ -250,7 +262,7 @@ iq8r_status iq8r_linear_partials(const int8_t* xq, int64_t m, const iq8r_weight*
   if (!aligned16(xq) || !aligned16(p)) return fail(IQ8R_ERR_INVALID_ARG, "%s: xq and p must be 16-byte aligned", fn);
   iq8r_weight sub = *w;
   sub.n = n1 - n0;
-  sub.codes = w->codes + n0 * w->k;
+  sub.codes = w->codes + n0 * (w->fmt == IQ8R_FMT_CB4_G128 ? w->k / 2 : w->k);
   // the partials need no scales, but the argument block carries valid ones
   if (w->fmt == IQ8R_FMT_G256_U8_BF16) {
     sub.sub_scale = w->sub_scale + n0 * (w->k / iq8r::kGroupTrunk);
@@ -273,6 +285,7 @@ iq8r_status iq8r_rescore(const int8_t* xq, const float* x_scale, int64_t m, cons
   if (n_cand < 0 || n_cand > 65535 * 32)
     return fail(IQ8R_ERR_INVALID_ARG, "%s: n_cand = %lld out of range", fn, (long long)n_cand);
   if (w->k > 48 * 1024) return fail(IQ8R_ERR_UNSUPPORTED, "%s: k above 49152 is not supported", fn);
+  if (w->fmt == IQ8R_FMT_CB4_G128) return fail(IQ8R_ERR_UNSUPPORTED, "%s: not for the codebook format", fn);
   if (m == 0 || n_cand == 0) return ok();
   if (!xq || !x_scale || !cand || !out_bf16) return fail(IQ8R_ERR_INVALID_ARG, "%s: NULL buffer", fn);
   if (!aligned16(xq)) return fail(IQ8R_ERR_INVALID_ARG, "%s: xq must be 16-byte aligned", fn);

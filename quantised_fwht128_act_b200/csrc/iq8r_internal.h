@@ -12,6 +12,9 @@ namespace iq8r {
 
 constexpr int kGroupTrunk = 256;  // u8 sub-scale block of the trunk format
 constexpr int kGroupHead = 128;   // bf16 scale block of the lm_head format
+// The drafter's 16-level codebook: a 4-bit index i stands for kCb4Table[i]
+// (the dflash recipe lines of the IQ8R page, "How this file was made").
+constexpr int kCb4Table[16] = {-127, -97, -75, -58, -43, -30, -18, -6, 6, 18, 30, 43, 58, 75, 97, 127};
 constexpr int kRot = 128;         // fwht128 acts on each 128 of K
 
 // Device error word values (0 = no error). The low byte names the wait.
@@ -60,6 +63,9 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_
 bool gemm_tc_supported(const LinearArgs& a, std::string* why);
 cudaError_t read_and_clear_device_error(uint32_t* err);
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
+// The drafter's codebook format (cb4_gemv.cuh): y or partials.
+cudaError_t launch_cb4(const LinearArgs& a, cudaStream_t stream);
+bool cb4_supported(int64_t k, std::string* why);
 // out[t][j] = y[t][cand[t][j]] (see rescore.cuh)
 cudaError_t launch_rescore(const LinearArgs& a, const int32_t* cand, int kc, uint16_t* out, cudaStream_t stream);
 

@@ -11,6 +11,7 @@
 #include "act_quant.cuh"
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
+#include "cb4_gemv.cuh"
 #include "rescore.cuh"
 #include "iq8r_device.cuh"
 #include "iq8r_internal.h"
@@ -520,6 +521,76 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_
                 : launch_tc_t<0, false, kTcMaxBM>(tw, tx, p, grid, stream);
   return part ? launch_tc_t<1, true, kTcMaxBM>(tw, tx, p, grid, stream)
               : launch_tc_t<1, false, kTcMaxBM>(tw, tx, p, grid, stream);
+}
+
+template <int MT, bool PARTIALS, int STEPS>
+cudaError_t launch_cb4_s(const LinearArgs& a, const DeviceInfo& d, cudaStream_t stream) {
+  auto kernel = cb4_gemv_kernel<MT, PARTIALS, STEPS>;
+  const int smem = MT * static_cast<int>(a.k);
+  static std::atomic<int> configured[kMaxDevices];
+  cudaError_t e = ensure_smem(kernel, smem, configured);
+  if (e != cudaSuccess) return e;
+  const int64_t rows_per_cta = kCb4Warps;
+  const int grid = static_cast<int>(std::min<int64_t>(d.num_sms, (a.n + rows_per_cta - 1) / rows_per_cta));
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pdl_config(dim3(grid), dim3(kCb4Warps * 32), static_cast<size_t>(smem), stream, attr);
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+// Row chunk of 4, 5 or 8 steps of 512 index bytes (K up to 4096, 5120 or
+// longer); the partial sums (tests) use the 8-step instance only.
+template <int MT, bool PARTIALS>
+cudaError_t launch_cb4_t(const LinearArgs& a, const DeviceInfo& d, cudaStream_t stream) {
+  const int64_t steps = (a.k / 2 + 511) / 512;
+  if constexpr (PARTIALS) {
+    return launch_cb4_s<MT, PARTIALS, 8>(a, d, stream);
+  } else {
+    if (steps > 5) return launch_cb4_s<MT, PARTIALS, 8>(a, d, stream);
+    if (steps == 5) return launch_cb4_s<MT, PARTIALS, 5>(a, d, stream);
+    return launch_cb4_s<MT, PARTIALS, 4>(a, d, stream);
+  }
+}
+
+// The codebook format: groups of up to 8 tokens a launch (their codes staged
+// in shared memory).
+cudaError_t launch_cb4(const LinearArgs& a, cudaStream_t stream) {
+  if (a.m == 0 || a.n == 0) return cudaSuccess;
+  DeviceInfo d;
+  cudaError_t e = device_info(&d);
+  if (e != cudaSuccess) return e;
+  const int64_t ng = a.k / kGroupHead;
+  for (int64_t m0 = 0; m0 < a.m; m0 += 8) {
+    const int mg = static_cast<int>(std::min<int64_t>(8, a.m - m0));
+    LinearArgs s = a;
+    s.m = mg;
+    s.xq = a.xq + m0 * a.k;
+    if (a.xs) s.xs = a.xs + m0;
+    if (a.y) s.y = a.y + m0 * a.n;
+    if (a.partials) s.partials = a.partials + m0 * a.n * ng;
+    const int mt = next_pow2(mg);
+    const bool part = a.partials != nullptr;
+    switch (mt) {
+      case 1: e = part ? launch_cb4_t<1, true>(s, d, stream) : launch_cb4_t<1, false>(s, d, stream); break;
+      case 2: e = part ? launch_cb4_t<2, true>(s, d, stream) : launch_cb4_t<2, false>(s, d, stream); break;
+      case 4: e = part ? launch_cb4_t<4, true>(s, d, stream) : launch_cb4_t<4, false>(s, d, stream); break;
+      default: e = part ? launch_cb4_t<8, true>(s, d, stream) : launch_cb4_t<8, false>(s, d, stream); break;
+    }
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+bool cb4_supported(int64_t k, std::string* why) {
+  DeviceInfo d;
+  if (device_info(&d) != cudaSuccess) {
+    if (why) *why = "cannot query the current device";
+    return false;
+  }
+  if (8 * k > d.smem_optin - kSmemReserve) {
+    if (why) *why = "k too large for the codebook kernel (8 tokens of codes must fit in shared memory)";
+    return false;
+  }
+  return true;
 }
 
 cudaError_t launch_rescore(const LinearArgs& a, const int32_t* cand, int kc, uint16_t* out, cudaStream_t stream) {

@@ -142,6 +142,32 @@ void pack_range(int fmt, bool rotate, int rule, const uint16_t* w, int64_t k, in
         const float d = s2 * s1;  // exact: 8-bit x 8-bit significands
         for (int64_t i = g * kGroupTrunk; i < (g + 1) * kGroupTrunk; ++i) out[i] = quantise(row[i], d);
       }
+    } else if (fmt == 2) {
+      // the drafter's codebook: nearest of 16 levels, two indices a byte
+      uint8_t* pk = reinterpret_cast<uint8_t*>(codes) + r * (k / 2);
+      for (int64_t g = 0; g < g128; ++g) {
+        float A = 0.0f;
+        for (int64_t i = g * kGroupHead; i < (g + 1) * kGroupHead; ++i) A = std::max(A, std::fabs(row[i]));
+        const uint16_t sb = bf16_round_up_bits(A / 127.0f);
+        scale[r * g128 + g] = sb;
+        const float s = bf16_to_float(sb);
+        for (int64_t i = g * kGroupHead; i < (g + 1) * kGroupHead; i += 2) {
+          uint8_t nib[2] = {8, 8};
+          for (int h = 0; h < 2; ++h) {
+            if (!(s > 0.0f)) continue;
+            const double t = static_cast<double>(row[i + h] / s);
+            double best = 1e300;
+            for (int c = 15; c >= 0; --c) {  // ties go to the larger level
+              const double d = std::fabs(t - static_cast<double>(kCb4Table[c]));
+              if (d < best) {
+                best = d;
+                nib[h] = static_cast<uint8_t>(c);
+              }
+            }
+          }
+          pk[i / 2] = static_cast<uint8_t>(nib[0] | (nib[1] << 4));
+        }
+      }
     } else {
       for (int64_t g = 0; g < g128; ++g) {
         float A = 0.0f;

@@ -49,7 +49,7 @@ def test_version(L):
 
 
 def test_packed_sizes_match_oracle(L):
-    for fmt in ("g256", "g128"):
+    for fmt in ("g256", "g128", "cb4"):
         for n, k in ((256, 512), (17408, 5120), (5120, 17408), (151936, 5120)):
             if fmt == "g256" and k % 256:
                 continue
@@ -197,3 +197,21 @@ def test_pack_rule_is_checked(L):
     scale = np.empty((2,), np.uint16)
     st = L.iq8r_pack_ex(0, 1, 7, w.ctypes.data, 2, 256, codes.ctypes.data, sub.ctypes.data, scale.ctypes.data, 1)
     assert st == iq8r.IQ8R_ERR_INVALID_ARG
+
+
+def test_pack_cb4_byte_identical_to_oracle(L):
+    """The drafter's codebook: indices and scales are the oracle's, on the
+    generator and on edge rows (zero, a spike, constants, tiny values)."""
+    _, w = gen_workload("decode", m=1, n=90, k=1024, seed=23)
+    w = w.copy()
+    w[3] = 0
+    w[4] = 0
+    w[4, 9] = f32_to_bf16_bits(np.array([-2.0], np.float32))[0]
+    w[5] = f32_to_bf16_bits(np.full(1024, 0.75, np.float32))
+    w[6] = f32_to_bf16_bits(np.full(1024, 1e-30, np.float32))
+    for rotate in (True, False):
+        codes, sub, scale = iq8r.iq8r_pack(w, "cb4", rotate)
+        p, s = oracle.pack_cb4(w, rotate)
+        assert sub is None and np.array_equal(codes, p) and np.array_equal(scale, s)
+    with pytest.raises(iq8r.IQ8RError):
+        iq8r.iq8r_pack(w, "cb4", True, rule="search")

@@ -479,3 +479,45 @@ def test_search_packed_weights(fmt, m, n, k, path):
     assert np.array_equal(gpu_partials(x, W, path=p), oracle.partials(q, codes, g))
     y64 = oracle.linear(q, a, fmt, codes, sub, scale, rotated=True)
     check_output(gpu_linear(x, W, path=p), y64, oracle.linear_bf16(y64))
+
+
+# ------------------------------------------ the drafter's 16-level codebook
+
+def _cb4_case(m, n, k, seed):
+    x, w = gen_workload("decode", m=m, n=n, k=k, seed=seed)
+    packed, scale = oracle.pack_cb4(w, True)
+    W = iq8r.IQ8RWeight.from_packed(packed, None, scale, "cb4", True)
+    return x, packed, scale, W
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 17408, 5120), (3, 1000, 768), (8, 300, 17408), (13, 77, 2560),
+                                   (2, 129, 128)])
+def test_cb4_partials_and_linear(m, n, k):
+    """Codebook format through its GEMV: exact per-128 partial sums of the
+    levels, and outputs within tolerance of the oracle; the tensor-core path
+    is refused."""
+    x, packed, scale, W = _cb4_case(m, n, k, seed=91 + m)
+    assert W.k == k
+    q, a = oracle.act_quant(x)
+    vals = oracle.decode_cb4(packed)
+    assert np.array_equal(gpu_partials(x, W), oracle.partials(q, vals, 128))
+    y64 = oracle.linear(q, a, "cb4", packed, None, scale, rotated=True)
+    check_output(gpu_linear(x, W), y64, oracle.linear_bf16(y64))
+    xq, xs = iq8r.iq8r_rotate_quant_act(dev_bf16(x))
+    with pytest.raises(iq8r.IQ8RError):
+        iq8r.iq8r_linear_ex(xq, xs, W, path=iq8r.IQ8R_PATH_TC)
+    # the whole layer from bf16 activations
+    y = iq8r.iq8r_linear_bf16(dev_bf16(x), W,
+                              xq_out=torch.empty(x.shape, dtype=torch.int8, device="cuda"),
+                              x_scale_out=torch.empty((m,), dtype=torch.float32, device="cuda"))
+    torch.cuda.synchronize()
+    check_output(host_bits(y), y64, oracle.linear_bf16(y64))
+    iq8r.iq8r_get_device_error()
+
+
+def test_cb4_partials_window():
+    x, packed, scale, W = _cb4_case(4, 600, 1024, seed=97)
+    q, _ = oracle.act_quant(x)
+    vals = oracle.decode_cb4(packed)
+    for n0, n1 in [(0, 5), (7, 300), (599, 600)]:
+        assert np.array_equal(gpu_partials(x, W, n0, n1), oracle.partials(q, vals[n0:n1], 128))

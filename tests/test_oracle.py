@@ -232,3 +232,48 @@ def test_pack_search_minimises_group_error(fmt):
             q = np.clip(np.rint(vals / np.float32(chosen)), -127, 127).astype(np.int8)
             assert np.array_equal(c1[r, b * g:(b + 1) * g], q)
     assert improved > 0
+
+
+# ------------------------------------------ the drafter's 16-level codebook
+
+def test_cb4_nearest_level_and_layout():
+    """Every index is the nearest codebook level to w'/s (ties to the larger
+    level), the scale covers the group's largest value, the error is at most
+    half the widest gap, and two indices share a byte, even K low."""
+    _, w = gen_workload("decode", m=1, n=5, k=384, seed=41)
+    packed, scale = oracle.pack_cb4(w, True)
+    wr = oracle.fwht128_f32(oracle.bf16_to_f32(w))
+    s = oracle.bf16_to_f32(scale)
+    table = [-127, -97, -75, -58, -43, -30, -18, -6, 6, 18, 30, 43, 58, 75, 97, 127]
+    vals = oracle.decode_cb4(packed)
+    for r in range(5):
+        for g in range(3):
+            sg = np.float32(s[r, g])
+            amax = np.max(np.abs(wr[r, g * 128:(g + 1) * 128]))
+            assert sg * 127 >= amax
+            for j in range(128):
+                kk = g * 128 + j
+                t = float(np.float32(wr[r, kk]) / sg)
+                best = min(table, key=lambda v: (abs(t - v), -v))
+                assert vals[r, kk] == best
+                assert abs(float(wr[r, kk]) - float(sg) * best) <= float(sg) * 15 + 1e-12
+                byte = packed[r, kk // 2]
+                nib = (byte & 0x0F) if kk % 2 == 0 else (byte >> 4)
+                assert table[nib] == vals[r, kk]
+
+
+def test_cb4_ties_and_zero_group():
+    """Hand-made groups: a value half way between two levels takes the larger
+    one (-112 -> -97, 0 -> +6); an all-zero group has scale 0 and index 8."""
+    s = 1.0
+    grp = np.zeros(128, np.float32)
+    grp[0] = 127.0 * s     # sets the scale to exactly 1 (bf16 of 127/127)
+    grp[1] = -112.0        # between -127 and -97
+    grp[2] = 0.0           # between -6 and +6
+    grp[3] = 36.5          # 6.5 from both 30 and 43: a tie -> 43
+    w = np.stack([grp, np.zeros(128, np.float32)])
+    packed, scale = oracle.pack_cb4(oracle.f32_to_bf16_exact(w), rotate=False)
+    v = oracle.decode_cb4(packed)
+    assert oracle.bf16_to_f32(scale)[0, 0] == 1.0
+    assert list(v[0, :4]) == [127, -97, 6, 43]
+    assert scale[1, 0] == 0 and np.all(packed[1] == 0x88)
