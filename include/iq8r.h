@@ -4,11 +4,13 @@
  * The layer, as the "radiance" model cards describe it:
  *
  *  - "Qwen3.8-27B IQ8R + DFlash2 -- radiance container", table row "Weights":
- *    every trunk linear is int8 with codes -127..127, a u8 scale per row and
- *    256 of K under a bf16 scale per row, each 128 of K rotated by the
- *    unnormalised Hadamard; the lm_head is int8 with a bf16 scale per row and
- *    128 of K.
- *  - same page, table row "Activations": int8 under the same rotation (W8A8).
+ *    the trunk linears hold int8 codes in -127..127 with one u8 scale for
+ *    every row and 256-wide block of K, below one bf16 scale per row, every
+ *    128 of K first rotated by a Hadamard transform without normalisation;
+ *    the lm_head holds int8 codes with one bf16 scale for every row and
+ *    128-wide block of K.
+ *  - same page, table row "Activations": the activations are int8 too, in
+ *    the same rotated domain (W8A8).
  *  - same page, "How this file was made": the recipe rules
  *    "codes=i8 group=256 scale=u8 scale2=bf16 block2=1x* transform=fwht128
  *    clamp=sym" (trunk) and "codes=i8 group=128 scale=bf16 clamp=sym"
@@ -116,16 +118,17 @@ iq8r_status iq8r_packed_sizes(int32_t fmt, int64_t n, int64_t k, size_t* codes_b
  *   sub_scale u8 [n][k/256] host (out; G256 only, NULL for G128)
  *   scale     bf16 [n] (G256) or [n][k/128] (G128) host (out)
  *   n_threads host threads to use; <= 0 picks the hardware concurrency.
- * Trunk: "a u8 scale per row and 256 of K under a bf16 scale a row" (IQ8R
- * page, "Weights"); lm_head: "a bf16 scale per row and 128" (same row).
+ * Trunk: a u8 scale for each row and 256 of K below a bf16 row scale (IQ8R
+ * page, "Weights"); lm_head: a bf16 scale for each row and 128 of K (same
+ * row).
  * Output is byte-identical to the stated definition in the file comment. */
 iq8r_status iq8r_pack(int32_t fmt, int32_t rotate, const uint16_t* w_bf16, int64_t n, int64_t k,
                       int8_t* codes, uint8_t* sub_scale, uint16_t* scale, int32_t n_threads);
 
 /* Packing rules: IQ8R_RULE_RTN is iq8r_pack's. IQ8R_RULE_SEARCH is the
- * recipes' "rule=search" ("a scale per 128 columns searched for least
- * error", "Qwen3.8-Flash-Next, IQR-V4 -- radiance container", row "Trunk"),
- * in this reading: per group, the RTN scale (the smallest that clips
+ * recipes' "rule=search" (one scale per 128 columns, chosen by a search for
+ * the least error: "Qwen3.8-Flash-Next, IQR-V4 -- radiance container", row
+ * "Trunk"), in this reading: per group, the RTN scale (the smallest that clips
  * nothing) and the 15 next smaller ones are tried, and the one with the least
  * sum of (w' - code * step)^2 over the group (in double, added in order)
  * is kept, ties going to the larger scale. For the trunk the candidates are
@@ -137,8 +140,8 @@ typedef enum { IQ8R_RULE_RTN = 0, IQ8R_RULE_SEARCH = 1 } iq8r_rule;
 iq8r_status iq8r_pack_ex(int32_t fmt, int32_t rotate, int32_t rule, const uint16_t* w_bf16, int64_t n,
                          int64_t k, int8_t* codes, uint8_t* sub_scale, uint16_t* scale, int32_t n_threads);
 
-/* Rotate and quantise activations: "int8 under the same rotation (W8A8)"
- * (IQ8R page, "Activations"), one fp32 scale per token.
+/* Rotate and quantise activations: int8 in the weights' rotated domain,
+ * W8A8 (IQ8R page, "Activations"), one fp32 scale per token.
  *   x_bf16  device bf16 [m][k], raw 16-bit patterns, 16-byte aligned
  *   m >= 0 (0 launches nothing), k % 128 == 0, 0 < k <= 2^30
  *   rotate  1: x' = T(x) in fp32; 0: x' = x

@@ -8,17 +8,19 @@ does, and the two share no code.
 What it follows (the pages are model cards of the "radiance" engine):
 
 * "Qwen3.8-27B IQ8R + DFlash2 -- radiance container", table row "Weights":
-  every trunk linear is int8 with codes -127..127, a u8 scale per row and
-  256 of K under a bf16 scale per row, each 128 of K rotated by the
-  unnormalised Hadamard; the lm_head is int8 with a bf16 scale per row and
-  128 of K.
-* same page, table row "Activations": int8 under the same rotation (W8A8).
+  the trunk linears hold int8 codes in -127..127 with one u8 scale for every
+  row and 256-wide block of K, below one bf16 scale per row; every 128 of K
+  is first rotated by a Hadamard transform that is not normalised. The
+  lm_head holds int8 codes with one bf16 scale for every row and 128-wide
+  block of K.
+* same page, table row "Activations": the activations are int8 too, in the
+  same rotated domain (W8A8).
 * same page, "How this file was made", the recipe rules
   ``codes=i8 group=256 scale=u8 scale2=bf16 block2=1x* transform=fwht128
   clamp=sym`` (trunk) and ``codes=i8 group=128 scale=bf16 clamp=sym``
   (lm_head).
 * "Qwen3.8-Flash-Next, IQR-V4 -- radiance container", row "Routed experts":
-  the transform is the 128-point Walsh-Hadamard rotation.
+  the rotation is a 128-point Walsh-Hadamard transform.
 
 Where the pages are silent the oracle writes down a stated definition (the
 library follows it exactly):
@@ -76,9 +78,9 @@ __all__ = [
     "rescore",
 ]
 
-GROUP_TRUNK = 256  # "a u8 scale per row and 256 of K" (IQ8R page, "Weights")
-GROUP_HEAD = 128   # "a bf16 scale per row and 128" (IQ8R page, "Weights")
-CODE_MAX = 127     # "codes -127..127", clamp=sym (IQ8R page, "Weights" and recipe)
+GROUP_TRUNK = 256  # trunk: one u8 scale per row and 256 of K (IQ8R page, "Weights")
+GROUP_HEAD = 128   # lm_head: one bf16 scale per row and 128 of K (IQ8R page, "Weights")
+CODE_MAX = 127     # codes in -127..127, clamp=sym (IQ8R page, "Weights" and recipe)
 SUB_MAX = 255      # largest u8 sub-scale (recipe: scale=u8)
 ROT = 128          # fwht128: the rotation acts on each 128 of K
 # The drafter's 16-level integer codebook (IQ8R page, "How this file was
@@ -146,9 +148,10 @@ def bf16_round_nearest(v: np.ndarray) -> np.ndarray:
 def hadamard128() -> np.ndarray:
     """The 128x128 unnormalised Hadamard matrix, natural (Sylvester) order.
 
-    H[i][j] = (-1) ** popcount(i & j): the "unnormalised Hadamard" of the
-    IQ8R page ("Weights") and the "128-point Walsh-Hadamard rotation" of the
-    Flash-Next page ("Routed experts"). No 1/sqrt(128) factor.
+    H[i][j] = (-1) ** popcount(i & j): the rotation of the IQ8R page
+    ("Weights"), a Hadamard transform without normalisation, which the
+    Flash-Next page ("Routed experts") names a 128-point Walsh-Hadamard
+    rotation. No 1/sqrt(128) factor.
     """
     i = np.arange(ROT)
     a = i[:, None] & i[None, :]
@@ -197,8 +200,8 @@ def fwht128_f64(v: np.ndarray) -> np.ndarray:
 def act_quant(x_bits: np.ndarray, rotate: bool = True):
     """Rotate and quantise activations to int8, one scale per token.
 
-    "int8 under the same rotation (W8A8)" (IQ8R page, "Activations"). The
-    granularity is not given; the stated definition is per token (row):
+    The activations are int8 in the weights' rotated domain, W8A8 (IQ8R page,
+    "Activations"). The granularity is not given; the stated definition is per token (row):
 
       x' = fwht128(x) in float32 (or x itself when ``rotate`` is false),
       amax = max |x'|, inv = 127 / amax (float32 divide),
@@ -360,8 +363,8 @@ def _group_sse(blocks: np.ndarray, d: np.ndarray) -> np.ndarray:
 def pack_search(w_bits: np.ndarray, fmt: str = "g256", rotate: bool = True, window: int = SEARCH_WINDOW):
     """The recipes' ``rule=search``: per group, the scale with least
     reconstruction error. "Qwen3.8-Flash-Next, IQR-V4 -- radiance
-    container", row "Trunk": "a scale per 128 columns searched for least
-    error"; the IQ8R recipe lines carry ``rule=search``.
+    container", row "Trunk", picks one scale per 128 columns by a search for
+    the least error; the IQ8R recipe lines carry ``rule=search``.
 
     Stated reading: start from the RTN scale of ``pack`` (the smallest that
     clips nothing) and try it and the ``window - 1`` next smaller ones --

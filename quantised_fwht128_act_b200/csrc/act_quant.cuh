@@ -1,6 +1,6 @@
-// Activation rotate + int8 quantise: "int8 under the same rotation (W8A8)"
-// ("Qwen3.8-27B IQ8R + DFlash2 -- radiance container", table row
-// "Activations"), one fp32 scale per token.
+// Activation rotate + int8 quantise: the activations are int8 in the same
+// rotated domain as the weights, W8A8 ("Qwen3.8-27B IQ8R + DFlash2 --
+// radiance container", table row "Activations"), one fp32 scale per token.
 //
 // One CTA per token row. A thread owns "slots" of 16 consecutive elements
 // (two 16-byte bf16 loads, one 16-byte int8 store). A 128-chunk is 8 slots

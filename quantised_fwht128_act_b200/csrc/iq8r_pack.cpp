@@ -4,7 +4,7 @@
 // "Weights", and the recipe rule "codes=i8 group=256 scale=u8 scale2=bf16
 // block2=1x* transform=fwht128 clamp=sym"): int8 codes -127..127, a u8
 // sub-scale per (row, 256 of K) under a bf16 scale per row, each 128 of K
-// rotated by the unnormalised Hadamard first.
+// rotated first by the Hadamard transform without normalisation.
 // lm_head (same row; recipe "codes=i8 group=128 scale=bf16 clamp=sym"): a
 // bf16 scale per (row, 128 of K).
 //
@@ -91,10 +91,10 @@ inline double group_sse(const float* v, int64_t len, float d) {
   return sse;
 }
 
-// The recipes' rule=search ("a scale per 128 columns searched for least
-// error", "Qwen3.8-Flash-Next, IQR-V4 -- radiance container", row "Trunk"):
-// the RTN step and the kSearchWindow - 1 next smaller ones, least error wins,
-// ties to the larger step.
+// The recipes' rule=search (one scale per 128 columns chosen by a search for
+// the least error: "Qwen3.8-Flash-Next, IQR-V4 -- radiance container", row
+// "Trunk"): the RTN step and the kSearchWindow - 1 next smaller ones, least
+// error wins, ties to the larger step.
 constexpr int kSearchWindow = 16;
 
 void pack_range(int fmt, bool rotate, int rule, const uint16_t* w, int64_t k, int64_t r0, int64_t r1,

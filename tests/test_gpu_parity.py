@@ -365,7 +365,7 @@ def test_tc_lm_head_format():
     check_output(gpu_linear(x, W, path=iq8r.IQ8R_PATH_TC), y64, oracle.linear_bf16(y64))
 
 
-# the trunk in the earlier IQ8R format (a bf16 scale per row and 128 of K):
+# the trunk in the earlier IQ8R format (one bf16 scale for each row and 128-wide block of K):
 # the lm_head kernels at trunk shapes, through both kernels
 @pytest.mark.parametrize("path", ["gemv", "tc"])
 @pytest.mark.parametrize("m,n,k", [(1, 17408, 5120), (16, 512, 17408), (300, 640, 5120)])
