@@ -79,7 +79,7 @@ __device__ __forceinline__ void cb4_rows_step(const LinearArgs& a, const int8_t*
     for (int i = 0; i < 4; ++i) cb4_decode8(wv[i], t0, t1, t2, t3, lv[2 * i], lv[2 * i + 1]);
     const int kk = valid ? 2 * o : 0;          // first weight of the lane's 32
     const int blk = kk / kGroupHead;           // the 32 share one 128-block
-    const float sb = bf16_bits_to_float(static_cast<uint16_t>(scl[u]));  // loaded with the codes
+    const float sb = valid ? bf16_bits_to_float(static_cast<uint16_t>(scl[u])) : 0.0f;  // loaded with the codes
 #pragma unroll
     for (int m = 0; m < MT; ++m) {
       const int4 x0 = *reinterpret_cast<const int4*>(act + m * K + kk);
@@ -127,14 +127,18 @@ __global__ void __launch_bounds__(kCb4Warps * 32, 1) cb4_gemv_kernel(const Linea
   const int64_t nw = static_cast<int64_t>(gridDim.x) * kCb4Warps;
 
   // a row chunk's codes and the scale of each lane's block, loaded together
-  // (a scale fetched only when needed would wait behind the weight stream)
+  // (a scale fetched only when needed would wait behind the weight stream).
+  // Within a row every lane loads unconditionally, lanes and steps past the
+  // row's end from its first bytes: the arithmetic masks them, and no select
+  // on a load's result makes the warp wait for the data it is prefetching.
   auto load = [&](int64_t row, int s0, int4 (&buf)[STEPS], uint32_t (&scl)[STEPS]) {
+    if (row >= N) return;  // warp-uniform; the slot is never computed
 #pragma unroll
     for (int u = 0; u < STEPS; ++u) {
-      const int o = (s0 + u) * 512 + lane * 16;
-      const bool v = row < N && s0 + u < nsteps && o < kb;
-      buf[u] = v ? __ldg(reinterpret_cast<const int4*>(codes + row * kb + o)) : make_int4(0, 0, 0, 0);
-      scl[u] = (v && !PARTIALS) ? static_cast<uint32_t>(__ldg(a.scale + row * ng + (2 * o) / kGroupHead)) : 0u;
+      int o = (s0 + u) * 512 + lane * 16;
+      o = o < kb ? o : 0;
+      buf[u] = __ldg(reinterpret_cast<const int4*>(codes + row * kb + o));
+      if (!PARTIALS) scl[u] = static_cast<uint32_t>(__ldg(a.scale + row * ng + (2 * o) / kGroupHead));
     }
   };
 
@@ -143,6 +147,14 @@ __global__ void __launch_bounds__(kCb4Warps * 32, 1) cb4_gemv_kernel(const Linea
   // out before waiting for the kernel that writes the activation codes
   int4 ring[DEPTH][STEPS];
   uint32_t rsc[DEPTH][STEPS];
+#pragma unroll
+  for (int d = 0; d < DEPTH; ++d) {
+#pragma unroll
+    for (int u = 0; u < STEPS; ++u) {
+      ring[d][u] = make_int4(0, 0, 0, 0);
+      rsc[d][u] = 0u;
+    }
+  }
   const bool whole = nsteps <= STEPS;
   if (whole) {
 #pragma unroll
