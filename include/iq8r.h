@@ -73,8 +73,9 @@ typedef enum {
    * "How this file was made", the dflash recipe lines), two a byte with the
    * even K position in the low nibble, and a bf16 scale per (row, 128 of K);
    * y as for G128 with the codes' levels. Packed by nearest level (ties to
-   * the larger) under s = bf16 of A / 127 rounded up. GEMV only (any M, 8
-   * tokens a launch); not for iq8r_rescore. */
+   * the larger) under s = bf16 of A / 127 rounded up (IQ8R_RULE_RTN) or the
+   * searched scale (IQ8R_RULE_SEARCH). GEMV only (any M, 8 tokens a launch);
+   * not for iq8r_rescore. */
   IQ8R_FMT_CB4_G128 = 2
 } iq8r_format;
 
@@ -132,8 +133,9 @@ iq8r_status iq8r_pack(int32_t fmt, int32_t rotate, const uint16_t* w_bf16, int64
  * nothing) and the 15 next smaller ones are tried, and the one with the least
  * sum of (w' - code * step)^2 over the group (in double, added in order)
  * is kept, ties going to the larger scale. For the trunk the candidates are
- * s1, s1 - 1, ... (>= 1) under the unchanged row scale s2; for G128 they are
- * s and the next smaller bf16 values. */
+ * s1, s1 - 1, ... (>= 1) under the unchanged row scale s2; for G128 and the
+ * codebook format they are s and the next smaller bf16 values, and for the
+ * codebook each value's term uses its nearest level at that scale. */
 typedef enum { IQ8R_RULE_RTN = 0, IQ8R_RULE_SEARCH = 1 } iq8r_rule;
 
 /* iq8r_pack with a packing rule (same arguments otherwise). */

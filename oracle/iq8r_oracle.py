@@ -36,7 +36,8 @@ library follows it exactly):
 * the factor 1/128 (H H = 128 I) is applied to the output.
 
 Also written here: ``pack_search`` (the recipes' rule=search: least-error
-scales among the RTN scale and the 15 below it), ``pack_cb4`` / ``decode_cb4``
+scales among the RTN scale and the 15 below it, for all three formats),
+``pack_cb4`` / ``decode_cb4``
 (the drafter's 16-level codebook: nearest level under s = bf16 of A / 127
 rounded up, ties to the larger level) and ``rescore`` (the layer at a list of
 candidate rows).
@@ -325,14 +326,23 @@ def pack_cb4(w_bits: np.ndarray, rotate: bool = True):
     idx = np.full((n, ng, GROUP_HEAD), 8, dtype=np.uint8)
     sz = s > 0
     if np.any(sz):
-        t = (blocks[sz] / s[sz][:, None]).astype(np.float64)        # [groups, 128]
-        dist = np.abs(t[..., None] - CB4_TABLE.astype(np.float64))  # [groups, 128, 16]
-        # least distance, ties to the larger level: search from the top index down
-        rev = dist[..., ::-1]
-        idx[sz] = (15 - np.argmin(rev, axis=-1)).astype(np.uint8)
-    idx = idx.reshape(n, k)
-    packed = (idx[:, 0::2] | (idx[:, 1::2] << 4)).astype(np.uint8)
-    return packed, f32_to_bf16_exact(s)
+        idx[sz] = _cb4_indices(blocks[sz], s[sz])
+    return _cb4_nibbles(idx.reshape(n, k)), f32_to_bf16_exact(s)
+
+
+def _cb4_indices(blocks: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """Index of the level nearest to w' / s for each value of blocks
+    [..., G] at scales s [...] (> 0): float32 quotient, float64 distances,
+    ties to the larger level."""
+    t = (blocks / s[..., None]).astype(np.float64)
+    dist = np.abs(t[..., None] - CB4_TABLE.astype(np.float64))  # [..., G, 16]
+    # least distance, ties to the larger level: search from the top index down
+    return (15 - np.argmin(dist[..., ::-1], axis=-1)).astype(np.uint8)
+
+
+def _cb4_nibbles(idx: np.ndarray) -> np.ndarray:
+    """Indices [N, K] -> bytes [N, K/2], the even K position in the low nibble."""
+    return (idx[:, 0::2] | (idx[:, 1::2] << 4)).astype(np.uint8)
 
 
 def decode_cb4(packed: np.ndarray) -> np.ndarray:
@@ -360,20 +370,34 @@ def _group_sse(blocks: np.ndarray, d: np.ndarray) -> np.ndarray:
     return np.cumsum(e * e, axis=-1)[..., -1]
 
 
+def _cb4_sse(blocks: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """Squared reconstruction error of each codebook group at scale s (> 0):
+    (w' - level * s) squared in float64, the levels those of
+    ``_cb4_indices``, the terms added left to right."""
+    lv = CB4_TABLE[_cb4_indices(blocks, s)].astype(np.float64)
+    e = blocks.astype(np.float64) - lv * s[..., None].astype(np.float64)
+    return np.cumsum(e * e, axis=-1)[..., -1]
+
+
 def pack_search(w_bits: np.ndarray, fmt: str = "g256", rotate: bool = True, window: int = SEARCH_WINDOW):
     """The recipes' ``rule=search``: per group, the scale with least
     reconstruction error. "Qwen3.8-Flash-Next, IQR-V4 -- radiance
     container", row "Trunk", picks one scale per 128 columns by a search for
-    the least error; the IQ8R recipe lines carry ``rule=search``.
+    the least error; the IQ8R recipe lines carry ``rule=search``, the trunk's
+    and the drafter's codebook lines alike.
 
     Stated reading: start from the RTN scale of ``pack`` (the smallest that
     clips nothing) and try it and the ``window - 1`` next smaller ones --
     trunk: s1, s1 - 1, ... (s1 >= 1) under the unchanged row scale s2;
-    lm_head: s and the next smaller bf16 values (> 0). Smaller steps clip the
-    group's largest values but refine the rest. The error of a candidate is
-    the sum of (w' - code * step)**2 over the group (``_group_sse``); the
-    least wins, ties go to the larger scale. Same returns as ``pack``.
+    lm_head and codebook: s and the next smaller bf16 values (> 0). Smaller
+    steps clip the group's largest values but refine the rest. The error of a
+    candidate is the sum of (w' - value * step)**2 over the group, the value
+    the code (``_group_sse``) or the nearest level (``_cb4_sse``); the least
+    wins, ties go to the larger scale. Same returns as ``pack`` (for "cb4":
+    packed indices, None, scales).
     """
+    if fmt == "cb4":
+        return _pack_search_cb4(w_bits, rotate, window)
     codes, sub, scale = pack(w_bits, fmt, rotate)
     w = bf16_to_f32(w_bits)
     n, k = w.shape
@@ -432,6 +456,40 @@ def pack_search(w_bits: np.ndarray, fmt: str = "g256", rotate: bool = True, wind
             codes[r0:r1] = q
         return codes.reshape(n, k), None, scale
     raise ValueError(fmt)
+
+
+def _pack_search_cb4(w_bits: np.ndarray, rotate: bool, window: int):
+    """``pack_search`` for the codebook format: the bf16 scale candidates of
+    the lm_head, scored by ``_cb4_sse``; the indices are those of the chosen
+    scale."""
+    _, scale = pack_cb4(w_bits, rotate)
+    w = bf16_to_f32(w_bits)
+    n, k = w.shape
+    wr = fwht128_f32(w) if rotate else w.copy()
+    ng = k // GROUP_HEAD
+    scale = scale.copy()
+    idx = np.full((n, ng, GROUP_HEAD), 8, dtype=np.uint8)
+    for r0 in range(0, n, 64):  # rows in chunks: the level distances take memory
+        r1 = min(n, r0 + 64)
+        blocks = wr[r0:r1].reshape(r1 - r0, ng, GROUP_HEAD)
+        b_rtn = scale[r0:r1].astype(np.int64)
+        best = np.full((r1 - r0, ng), np.inf)
+        best_b = b_rtn.copy()
+        for i in range(window):
+            b = b_rtn - i
+            ok = (b_rtn > 0) & (b >= 1)  # positive bf16 bit patterns: one step down is the next smaller value
+            s = bf16_to_f32(np.where(ok, b, 0x3F80).astype(np.uint16))
+            sse = _cb4_sse(blocks, s)
+            better = ok & (sse < best)
+            best = np.where(better, sse, best)
+            best_b = np.where(better, b, best_b)
+        scale[r0:r1] = best_b.astype(np.uint16)
+        s = bf16_to_f32(scale[r0:r1])
+        sz = s > 0
+        if np.any(sz):
+            sub_idx = idx[r0:r1]
+            sub_idx[sz] = _cb4_indices(blocks[sz], s[sz])
+    return _cb4_nibbles(idx.reshape(n, k)), None, scale
 
 
 # ------------------------------------------------------------------ linear

@@ -166,8 +166,6 @@ iq8r_status iq8r_pack_ex(int32_t fmt, int32_t rotate, int32_t rule, const uint16
     return fail(IQ8R_ERR_INVALID_ARG, "%s: unknown rule %d", fn, rule);
   if (fmt != IQ8R_FMT_G256_U8_BF16 && fmt != IQ8R_FMT_G128_BF16 && fmt != IQ8R_FMT_CB4_G128)
     return fail(IQ8R_ERR_INVALID_ARG, "%s: unknown format %d", fn, fmt);
-  if (fmt == IQ8R_FMT_CB4_G128 && rule != IQ8R_RULE_RTN)
-    return fail(IQ8R_ERR_UNSUPPORTED, "%s: the codebook format packs by nearest level only", fn);
   if (rotate != 0 && rotate != 1) return fail(IQ8R_ERR_INVALID_ARG, "%s: rotate must be 0 or 1", fn);
   const int64_t g = fmt == IQ8R_FMT_G256_U8_BF16 ? iq8r::kGroupTrunk : iq8r::kGroupHead;
   if (n < 0 || k <= 0 || k % g)

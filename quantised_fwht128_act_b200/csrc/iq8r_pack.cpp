@@ -91,6 +91,34 @@ inline double group_sse(const float* v, int64_t len, float d) {
   return sse;
 }
 
+// Index of the codebook level nearest to w / s (s > 0): the quotient in
+// float32, the distances in double, ties going to the larger level.
+inline uint8_t cb4_index(float w, float s) {
+  const double t = static_cast<double>(w / s);
+  double best = 1e300;
+  uint8_t bi = 8;
+  for (int c = 15; c >= 0; --c) {  // from the top: a tie keeps the larger level
+    const double d = std::fabs(t - static_cast<double>(kCb4Table[c]));
+    if (d < best) {
+      best = d;
+      bi = static_cast<uint8_t>(c);
+    }
+  }
+  return bi;
+}
+
+// Squared reconstruction error of one codebook group at scale `s`:
+// (w' - level * s)^2 in double, added in index order.
+inline double cb4_sse(const float* v, int64_t len, float s) {
+  double sse = 0.0;
+  for (int64_t i = 0; i < len; ++i) {
+    const double e = static_cast<double>(v[i]) - static_cast<double>(kCb4Table[cb4_index(v[i], s)]) *
+                                                     static_cast<double>(s);
+    sse += e * e;
+  }
+  return sse;
+}
+
 // The recipes' rule=search (one scale per 128 columns chosen by a search for
 // the least error: "Qwen3.8-Flash-Next, IQR-V4 -- radiance container", row
 // "Trunk"): the RTN step and the kSearchWindow - 1 next smaller ones, least
@@ -148,24 +176,27 @@ void pack_range(int fmt, bool rotate, int rule, const uint16_t* w, int64_t k, in
       for (int64_t g = 0; g < g128; ++g) {
         float A = 0.0f;
         for (int64_t i = g * kGroupHead; i < (g + 1) * kGroupHead; ++i) A = std::max(A, std::fabs(row[i]));
-        const uint16_t sb = bf16_round_up_bits(A / 127.0f);
+        uint16_t sb = bf16_round_up_bits(A / 127.0f);
+        if (rule == 1 && sb > 0) {
+          const float* v = row.data() + g * kGroupHead;
+          double best = cb4_sse(v, kGroupHead, bf16_to_float(sb));
+          uint16_t best_b = sb;
+          for (int i = 1; i < kSearchWindow && static_cast<int>(sb) - i >= 1; ++i) {
+            const uint16_t c = static_cast<uint16_t>(sb - i);  // the next smaller positive bf16
+            const double e = cb4_sse(v, kGroupHead, bf16_to_float(c));
+            if (e < best) {
+              best = e;
+              best_b = c;
+            }
+          }
+          sb = best_b;
+        }
         scale[r * g128 + g] = sb;
         const float s = bf16_to_float(sb);
         for (int64_t i = g * kGroupHead; i < (g + 1) * kGroupHead; i += 2) {
-          uint8_t nib[2] = {8, 8};
-          for (int h = 0; h < 2; ++h) {
-            if (!(s > 0.0f)) continue;
-            const double t = static_cast<double>(row[i + h] / s);
-            double best = 1e300;
-            for (int c = 15; c >= 0; --c) {  // ties go to the larger level
-              const double d = std::fabs(t - static_cast<double>(kCb4Table[c]));
-              if (d < best) {
-                best = d;
-                nib[h] = static_cast<uint8_t>(c);
-              }
-            }
-          }
-          pk[i / 2] = static_cast<uint8_t>(nib[0] | (nib[1] << 4));
+          const uint8_t lo = s > 0.0f ? cb4_index(row[i], s) : 8;
+          const uint8_t hi = s > 0.0f ? cb4_index(row[i + 1], s) : 8;
+          pk[i / 2] = static_cast<uint8_t>(lo | (hi << 4));
         }
       }
     } else {

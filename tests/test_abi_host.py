@@ -200,8 +200,9 @@ def test_pack_rule_is_checked(L):
 
 
 def test_pack_cb4_byte_identical_to_oracle(L):
-    """The drafter's codebook: indices and scales are the oracle's, on the
-    generator and on edge rows (zero, a spike, constants, tiny values)."""
+    """The drafter's codebook: indices and scales are the oracle's, for both
+    rules, on the generator and on edge rows (zero, a spike, constants, tiny
+    values)."""
     _, w = gen_workload("decode", m=1, n=90, k=1024, seed=23)
     w = w.copy()
     w[3] = 0
@@ -213,5 +214,7 @@ def test_pack_cb4_byte_identical_to_oracle(L):
         codes, sub, scale = iq8r.iq8r_pack(w, "cb4", rotate)
         p, s = oracle.pack_cb4(w, rotate)
         assert sub is None and np.array_equal(codes, p) and np.array_equal(scale, s)
-    with pytest.raises(iq8r.IQ8RError):
-        iq8r.iq8r_pack(w, "cb4", True, rule="search")
+        codes, sub, scale = iq8r.iq8r_pack(w, "cb4", rotate, rule="search")
+        p, s_none, s = oracle.pack_search(w, "cb4", rotate)
+        assert sub is None and s_none is None
+        assert np.array_equal(codes, p) and np.array_equal(scale, s)

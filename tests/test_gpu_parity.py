@@ -515,6 +515,22 @@ def test_cb4_partials_and_linear(m, n, k):
     iq8r.iq8r_get_device_error()
 
 
+@pytest.mark.parametrize("m,n,k", [(1, 257, 5120), (5, 333, 1024)])
+def test_cb4_search_packed(m, n, k):
+    """Codebook weights packed by the C++ rule=search: the bytes are the
+    oracle's search result, the partial sums exact and the outputs within
+    tolerance."""
+    x, w = gen_workload("decode", m=m, n=n, k=k, seed=61 + m)
+    packed, sub, scale = iq8r.iq8r_pack(w, "cb4", True, rule="search")
+    want = oracle.pack_search(w, "cb4", True)
+    assert sub is None and np.array_equal(packed, want[0]) and np.array_equal(scale, want[2])
+    W = iq8r.IQ8RWeight.from_packed(packed, None, scale, "cb4", True)
+    q, a = oracle.act_quant(x)
+    assert np.array_equal(gpu_partials(x, W), oracle.partials(q, oracle.decode_cb4(packed), 128))
+    y64 = oracle.linear(q, a, "cb4", packed, None, scale, rotated=True)
+    check_output(gpu_linear(x, W), y64, oracle.linear_bf16(y64))
+
+
 def test_cb4_partials_window():
     x, packed, scale, W = _cb4_case(4, 600, 1024, seed=97)
     q, _ = oracle.act_quant(x)

@@ -234,6 +234,51 @@ def test_pack_search_minimises_group_error(fmt):
     assert improved > 0
 
 
+def _exact_cb4_sse(vals, scale):
+    """Exact (rational) squared error of a codebook group at a scale, each
+    value at its nearest level (brute force over the 16, ties to the larger)."""
+    from fractions import Fraction
+    table = [-127, -97, -75, -58, -43, -30, -18, -6, 6, 18, 30, 43, 58, 75, 97, 127]
+    tot = Fraction(0)
+    st = Fraction(float(scale))
+    for v in vals:
+        t = float(np.float32(v) / np.float32(scale))
+        lv = min(table, key=lambda c: (abs(t - c), -c))
+        e = Fraction(float(v)) - lv * st
+        tot += e * e
+    return tot
+
+
+def test_pack_search_cb4_minimises_group_error():
+    """Brute force for the codebook format: per group, the searched bf16
+    scale has the least exact squared error among the RTN scale and the 15
+    next smaller bf16 values, never does worse than RTN, does better on some
+    groups, and every index is the nearest level at the chosen scale."""
+    _, w = gen_workload("decode", m=1, n=4, k=256, seed=35)
+    wr = oracle.fwht128_f32(oracle.bf16_to_f32(w))
+    _, sc0 = oracle.pack_cb4(w, True)
+    p1, sub1, sc1 = oracle.pack_search(w, "cb4", True)
+    assert sub1 is None
+    table = [-127, -97, -75, -58, -43, -30, -18, -6, 6, 18, 30, 43, 58, 75, 97, 127]
+    vals1 = oracle.decode_cb4(p1)
+    improved = 0
+    for r in range(w.shape[0]):
+        for b in range(w.shape[1] // 128):
+            vals = wr[r, b * 128:(b + 1) * 128]
+            base = int(sc0[r, b])
+            cands = [oracle.bf16_to_f32(np.array([base - i], np.uint16))[0] for i in range(16) if base - i >= 1]
+            chosen = oracle.bf16_to_f32(sc1[r:r + 1, b])[0]
+            errs = [_exact_cb4_sse(vals, c) for c in cands]
+            e_chosen = _exact_cb4_sse(vals, chosen)
+            assert float(e_chosen) <= float(min(errs)) * (1 + 1e-9)
+            assert e_chosen <= errs[0]
+            improved += e_chosen < errs[0]
+            for j in range(128):
+                t = float(np.float32(vals[j]) / np.float32(chosen))
+                assert vals1[r, b * 128 + j] == min(table, key=lambda c: (abs(t - c), -c))
+    assert improved > 0
+
+
 # ------------------------------------------ the drafter's 16-level codebook
 
 def test_cb4_nearest_level_and_layout():

@@ -150,3 +150,12 @@ def test_search_with_a_misplaced_step_is_caught(monkeypatch):
     monkeypatch.setattr(om, "_group_sse", lambda blocks, d: real(blocks, d * np.float32(1.01)))
     with pytest.raises(AssertionError):
         test_oracle.test_pack_search_minimises_group_error("g256")
+
+
+def test_cb4_search_keeping_the_worst_scale_is_caught(monkeypatch):
+    """The codebook's rule=search that keeps the largest error."""
+    import test_oracle
+    real = om._cb4_sse
+    monkeypatch.setattr(om, "_cb4_sse", lambda blocks, s: -real(blocks, s))
+    with pytest.raises(AssertionError):
+        test_oracle.test_pack_search_cb4_minimises_group_error()
