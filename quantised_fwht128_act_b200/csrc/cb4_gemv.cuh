@@ -41,18 +41,20 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 }
 
 // 8 indices (one word, index j in bits 4j..4j+3) -> 8 int8 levels (2 words).
+// A permute reads only the low 16 bits of its selector, so one mask of the
+// whole word gives the selectors of indices 0-3 and, shifted, of 4-7.
 __device__ __forceinline__ void cb4_decode8(uint32_t w, uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3,
                                             uint32_t& out0, uint32_t& out1) {
   const uint32_t w4 = w << 4;
+  const uint32_t sel = w & 0x77777777u;  // the low 3 bits of every index
   // indices 0-3
-  const uint32_t s0 = w & 0x7777u;
-  const uint32_t lo0 = prmt(t0, t1, s0), hi0 = prmt(t2, t3, s0);
+  const uint32_t lo0 = prmt(t0, t1, sel), hi0 = prmt(t2, t3, sel);
   // byte k = 0xFF where index k has bit 3 set: the sign-replicate selectors
   // read bit 3 of index 2j from (w << 4) and of index 2j + 1 from w
   const uint32_t m0 = prmt(w4, w, 0xD9C8u);
   out0 = (lo0 & ~m0) | (hi0 & m0);
   // indices 4-7
-  const uint32_t s1 = (w >> 16) & 0x7777u;
+  const uint32_t s1 = sel >> 16;
   const uint32_t lo1 = prmt(t0, t1, s1), hi1 = prmt(t2, t3, s1);
   const uint32_t m1 = prmt(w4, w, 0xFBEAu);
   out1 = (lo1 & ~m1) | (hi1 & m1);
@@ -60,8 +62,9 @@ __device__ __forceinline__ void cb4_decode8(uint32_t w, uint32_t t0, uint32_t t1
 
 // One row chunk of STEPS x 512 index bytes (lane: STEPS x 16 bytes) against
 // the staged activation codes: per-block partial sums (PARTIALS) or the fp32
-// sum of s * P into facc.
-template <int MT, bool PARTIALS, int STEPS>
+// sum of s * P into facc. EXACT: every chunk is full (K / 2 a multiple of
+// STEPS x 512), so no lane is past the row's end.
+template <int MT, bool PARTIALS, int STEPS, bool EXACT>
 __device__ __forceinline__ void cb4_rows_step(const LinearArgs& a, const int8_t* act, const int4 (&buf)[STEPS],
                                               const uint32_t (&scl)[STEPS],
                                               int64_t row, int s0, int nsteps, int kb, int K, int M, int64_t N,
@@ -71,7 +74,7 @@ __device__ __forceinline__ void cb4_rows_step(const LinearArgs& a, const int8_t*
   for (int u = 0; u < STEPS; ++u) {
     if (s0 + u >= nsteps) break;               // warp-uniform
     const int o = (s0 + u) * 512 + lane * 16;  // index bytes; weights 2 * o ..
-    const bool valid = o < kb;                 // whole 4-lane blocks in or out (kb % 64 == 0)
+    const bool valid = EXACT || o < kb;        // whole 4-lane blocks in or out (kb % 64 == 0)
     const uint32_t wv[4] = {static_cast<uint32_t>(buf[u].x), static_cast<uint32_t>(buf[u].y),
                             static_cast<uint32_t>(buf[u].z), static_cast<uint32_t>(buf[u].w)};
     uint32_t lv[8];
@@ -108,8 +111,9 @@ __device__ __forceinline__ void cb4_rows_step(const LinearArgs& a, const int8_t*
 // Rows of at most STEPS x 512 index bytes are kept DEPTH rows ahead in
 // registers (a warp's rows: gw, gw + nw, ...): the row computed now was
 // loaded DEPTH - 1 rows earlier. Longer rows (STEPS chunks each) go one chunk
-// ahead.
-template <int MT, bool PARTIALS, int STEPS>
+// ahead. EXACT: K / 2 is a multiple of STEPS x 512, so every chunk is full and
+// the masks and clamps drop out.
+template <int MT, bool PARTIALS, int STEPS, bool EXACT>
 __global__ void __launch_bounds__(kCb4Warps * 32, 1) cb4_gemv_kernel(const LinearArgs a) {
   constexpr int DEPTH = STEPS <= 5 ? 3 : 2;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -136,7 +140,7 @@ __global__ void __launch_bounds__(kCb4Warps * 32, 1) cb4_gemv_kernel(const Linea
 #pragma unroll
     for (int u = 0; u < STEPS; ++u) {
       int o = (s0 + u) * 512 + lane * 16;
-      o = o < kb ? o : 0;
+      if (!EXACT) o = o < kb ? o : 0;
       buf[u] = __ldg(reinterpret_cast<const int4*>(codes + row * kb + o));
       if (!PARTIALS) scl[u] = static_cast<uint32_t>(__ldg(a.scale + row * ng + (2 * o) / kGroupHead));
     }
@@ -190,8 +194,8 @@ __global__ void __launch_bounds__(kCb4Warps * 32, 1) cb4_gemv_kernel(const Linea
         float facc[MT];
 #pragma unroll
         for (int m = 0; m < MT; ++m) facc[m] = 0.0f;
-        cb4_rows_step<MT, PARTIALS, STEPS>(a, act, ring[d], rsc[d], row, 0, nsteps, kb, K, M, N, ng, lane, t0, t1,
-                                          t2, t3, facc);
+        cb4_rows_step<MT, PARTIALS, STEPS, EXACT>(a, act, ring[d], rsc[d], row, 0, nsteps, kb, K, M, N, ng, lane,
+                                                 t0, t1, t2, t3, facc);
         load(row + DEPTH * nw, 0, ring[d], rsc[d]);  // this slot's next row
         finish(row, facc);
       }
@@ -205,12 +209,12 @@ __global__ void __launch_bounds__(kCb4Warps * 32, 1) cb4_gemv_kernel(const Linea
       load(row, 0, ring[0], rsc[0]);
       for (int s0 = 0; s0 < nsteps; s0 += 2 * STEPS) {
         if (s0 + STEPS < nsteps) load(row, s0 + STEPS, ring[1], rsc[1]);
-        cb4_rows_step<MT, PARTIALS, STEPS>(a, act, ring[0], rsc[0], row, s0, nsteps, kb, K, M, N, ng, lane, t0, t1,
-                                          t2, t3, facc);
+        cb4_rows_step<MT, PARTIALS, STEPS, EXACT>(a, act, ring[0], rsc[0], row, s0, nsteps, kb, K, M, N, ng, lane,
+                                                 t0, t1, t2, t3, facc);
         if (s0 + STEPS >= nsteps) break;
         if (s0 + 2 * STEPS < nsteps) load(row, s0 + 2 * STEPS, ring[0], rsc[0]);
-        cb4_rows_step<MT, PARTIALS, STEPS>(a, act, ring[1], rsc[1], row, s0 + STEPS, nsteps, kb, K, M, N, ng, lane,
-                                          t0, t1, t2, t3, facc);
+        cb4_rows_step<MT, PARTIALS, STEPS, EXACT>(a, act, ring[1], rsc[1], row, s0 + STEPS, nsteps, kb, K, M, N, ng,
+                                                 lane, t0, t1, t2, t3, facc);
       }
       finish(row, facc);
     }

@@ -523,9 +523,9 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_
               : launch_tc_t<1, false, kTcMaxBM>(tw, tx, p, grid, stream);
 }
 
-template <int MT, bool PARTIALS, int STEPS>
+template <int MT, bool PARTIALS, int STEPS, bool EXACT>
 cudaError_t launch_cb4_s(const LinearArgs& a, const DeviceInfo& d, cudaStream_t stream) {
-  auto kernel = cb4_gemv_kernel<MT, PARTIALS, STEPS>;
+  auto kernel = cb4_gemv_kernel<MT, PARTIALS, STEPS, EXACT>;
   const int smem = MT * static_cast<int>(a.k);
   static std::atomic<int> configured[kMaxDevices];
   cudaError_t e = ensure_smem(kernel, smem, configured);
@@ -538,16 +538,23 @@ cudaError_t launch_cb4_s(const LinearArgs& a, const DeviceInfo& d, cudaStream_t 
 }
 
 // Row chunk of 4, 5 or 8 steps of 512 index bytes (K up to 4096, 5120 or
-// longer); the partial sums (tests) use the 8-step instance only.
+// longer), the exact instance when K / 2 is a multiple of the chunk; the
+// partial sums (tests) use the general 8-step instance only.
+template <int MT, bool PARTIALS, int STEPS>
+cudaError_t launch_cb4_e(const LinearArgs& a, const DeviceInfo& d, cudaStream_t stream) {
+  if ((a.k / 2) % (STEPS * 512) == 0) return launch_cb4_s<MT, PARTIALS, STEPS, true>(a, d, stream);
+  return launch_cb4_s<MT, PARTIALS, STEPS, false>(a, d, stream);
+}
+
 template <int MT, bool PARTIALS>
 cudaError_t launch_cb4_t(const LinearArgs& a, const DeviceInfo& d, cudaStream_t stream) {
   const int64_t steps = (a.k / 2 + 511) / 512;
   if constexpr (PARTIALS) {
-    return launch_cb4_s<MT, PARTIALS, 8>(a, d, stream);
+    return launch_cb4_s<MT, PARTIALS, 8, false>(a, d, stream);
   } else {
-    if (steps > 5) return launch_cb4_s<MT, PARTIALS, 8>(a, d, stream);
-    if (steps == 5) return launch_cb4_s<MT, PARTIALS, 5>(a, d, stream);
-    return launch_cb4_s<MT, PARTIALS, 4>(a, d, stream);
+    if (steps > 5) return launch_cb4_e<MT, PARTIALS, 8>(a, d, stream);
+    if (steps == 5) return launch_cb4_e<MT, PARTIALS, 5>(a, d, stream);
+    return launch_cb4_e<MT, PARTIALS, 4>(a, d, stream);
   }
 }
 

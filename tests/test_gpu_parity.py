@@ -491,11 +491,13 @@ def _cb4_case(m, n, k, seed):
 
 
 @pytest.mark.parametrize("m,n,k", [(1, 17408, 5120), (3, 1000, 768), (8, 300, 17408), (13, 77, 2560),
-                                   (2, 129, 128)])
+                                   (2, 129, 128), (4, 100, 4096), (6, 200, 8192), (2, 150, 16384)])
 def test_cb4_partials_and_linear(m, n, k):
     """Codebook format through its GEMV: exact per-128 partial sums of the
     levels, and outputs within tolerance of the oracle; the tensor-core path
-    is refused."""
+    is refused. K = 5120, 4096, 8192 and 16384 take the instances for full
+    chunks (one chunk of 5, 4 or 8 steps; two chunks of 8), the rest the
+    general ones."""
     x, packed, scale, W = _cb4_case(m, n, k, seed=91 + m)
     assert W.k == k
     q, a = oracle.act_quant(x)
