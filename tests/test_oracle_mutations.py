@@ -159,3 +159,38 @@ def test_cb4_search_keeping_the_worst_scale_is_caught(monkeypatch):
     monkeypatch.setattr(om, "_cb4_sse", lambda blocks, s: -real(blocks, s))
     with pytest.raises(AssertionError):
         test_oracle.test_pack_search_cb4_minimises_group_error()
+
+
+def test_cb4_swapped_nibbles_are_caught(monkeypatch):
+    """The codebook's two indices a byte in the other order."""
+    import test_oracle
+    monkeypatch.setattr(om, "_cb4_nibbles", lambda idx: (idx[:, 1::2] | (idx[:, 0::2] << 4)).astype(np.uint8))
+    with pytest.raises(AssertionError):
+        test_oracle.test_cb4_nearest_level_and_layout()
+
+
+def test_cb4_ties_to_the_smaller_level_are_caught(monkeypatch):
+    """The codebook's nearest level with ties going down instead of up."""
+    import test_oracle
+
+    def ties_down(blocks, s):
+        t = (blocks / s[..., None]).astype(np.float64)
+        return np.argmin(np.abs(t[..., None] - om.CB4_TABLE.astype(np.float64)), axis=-1).astype(np.uint8)
+
+    monkeypatch.setattr(om, "_cb4_indices", ties_down)
+    with pytest.raises(AssertionError):
+        test_oracle.test_cb4_ties_and_zero_group()
+
+
+def test_rescore_of_the_neighbouring_row_is_caught(monkeypatch):
+    """Rescoring that gathers the row after each candidate."""
+    import test_oracle
+    real = om.rescore
+
+    def next_row(xq, a, fmt, codes, sub, scale_bits, cand, rotated=True):
+        c = np.minimum(np.asarray(cand) + 1, np.asarray(codes).shape[0] - 1)
+        return real(xq, a, fmt, codes, sub, scale_bits, c, rotated)
+
+    monkeypatch.setattr(oracle, "rescore", next_row)
+    with pytest.raises(AssertionError):
+        test_oracle.test_rescore_is_the_linear_at_the_candidates("g256")
