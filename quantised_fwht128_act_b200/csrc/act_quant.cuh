@@ -16,6 +16,7 @@ namespace iq8r {
 
 constexpr int kActSlot = 16;           // elements per slot
 constexpr int kActRegMaxK = 16384;     // register path up to this K
+constexpr int kActRegMaxThreads = 256;  // its CTA size limit (8 slots a thread cover K = 16384)
 constexpr int kActTwoPassThreads = 256;
 
 __device__ __forceinline__ void act_load_slot(const uint16_t* p, float (&v)[kActSlot], bool streaming) {
@@ -94,7 +95,7 @@ __device__ __forceinline__ float act_block_max(float v, float* red) {
 
 // K <= kActRegMaxK: the row stays in registers (J slots per thread).
 template <int J>
-__global__ void __launch_bounds__(128) act_quant_reg_kernel(const uint16_t* __restrict__ x, int k, int rotate,
+__global__ void __launch_bounds__(kActRegMaxThreads) act_quant_reg_kernel(const uint16_t* __restrict__ x, int k, int rotate,
                                                             int8_t* __restrict__ xq, float* __restrict__ xs) {
   __shared__ float red[32];
   pdl_launch_dependents();  // the next kernel may start its set-up

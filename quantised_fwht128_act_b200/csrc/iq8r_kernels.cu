@@ -217,8 +217,20 @@ cudaError_t launch_act_quant(const uint16_t* x, int64_t m, int64_t k, int rotate
     }
   }
   if (k <= kActRegMaxK) {
-    const int threads = slots <= 128 ? ((slots + 31) / 32) * 32 : 128;
-    const int j = (slots + threads - 1) / threads;
+    // J slots a thread, the CTA a multiple of 32 threads (at most
+    // kActRegMaxThreads): the choice with the fewest idle slots, which still
+    // run the butterflies and shuffles (K = 5120: 2 x 160, not 3 x 128)
+    int j = 0, threads = 0;
+    int64_t idle = -1;
+    for (int jj = 1; jj <= 8; ++jj) {
+      const int t = ((slots + jj - 1) / jj + 31) / 32 * 32;
+      const int64_t w = static_cast<int64_t>(jj) * t - slots;
+      if (t <= kActRegMaxThreads && (idle < 0 || w < idle)) {
+        j = jj;
+        threads = t;
+        idle = w;
+      }
+    }
     const int kk = static_cast<int>(k);
     switch (j) {
       case 1: act_quant_reg_kernel<1><<<grid, threads, 0, stream>>>(x, kk, rotate, xq, xs); break;

@@ -74,7 +74,8 @@ def test_act_bit_exact_prefill_full():
 # small M: a row spread over a cluster of CTAs; M >= 148: one CTA a row, the
 # row in registers up to K = 16384, two passes above
 @pytest.mark.parametrize("m,k", [(5, 128), (3, 640), (7, 2176), (1, 16384), (2, 16512), (3, 33024), (33, 1152),
-                                 (16, 17408), (147, 256), (148, 5120), (160, 16512)])
+                                 (16, 17408), (147, 256), (148, 5120), (160, 16512), (149, 768), (150, 2560),
+                                 (152, 1152), (200, 4096), (300, 16384)])
 def test_act_bit_exact_ragged_shapes(m, k):
     x, _ = gen_workload("decode", m=m, n=8, k=k, seed=m * 1000 + k)
     assert_act_exact(x)
