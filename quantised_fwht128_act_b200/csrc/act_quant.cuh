@@ -6,8 +6,9 @@
 // (two 16-byte bf16 loads, one 16-byte int8 store). A 128-chunk is 8 slots
 // held by 8 consecutive lanes, so fwht128's seven butterfly stages run as
 // h = 1, 2, 4, 8 inside the thread and h = 16, 32, 64 across lanes (xor 1,
-// 2, 4), in that order, each an IEEE add or subtract: the result is
-// bit-identical to the sequential radix-2 transform.
+// 2, 4; or, in the one-CTA-a-row kernel, through a shared-memory exchange),
+// in that order, each an IEEE add or subtract: the result is bit-identical
+// to the sequential radix-2 transform.
 #pragma once
 
 #include "iq8r_device.cuh"
@@ -62,6 +63,94 @@ __device__ __forceinline__ void act_fwht_slot(float (&v)[kActSlot], int lane) {
   }
 }
 
+// The same transform with h = 16, 32, 64 through shared memory instead of
+// shuffles. After the in-thread stages, each 8-lane group (one 128-chunk,
+// lane q holding elements 16q..16q+15) exchanges its chunk so that lane q
+// holds elements 16p + 2q + b (p = 0..7, b = 0, 1) as t[2p + b]; h = 16, 32,
+// 64 are then register butterflies over p with strides 1, 2, 4, in that
+// order, each the same add or subtract. Layout of a group's 128 floats:
+// element 16p + i at 8i + 4(i / 4) + p, groups kActXStride floats apart, so
+// the scalar writes (fixed i, the warp's 32 lanes) and the 16-byte reads
+// (fixed offset, 8 lanes a phase) fall in distinct banks. xb: the warp's
+// 4 * kActXStride floats, 16-byte aligned.
+constexpr int kActXStride = 152;  // floats a group (128 + 24; 152 = 24 mod 32)
+constexpr int kActCStride = 144;  // bytes a group of codes (128 + 16)
+
+__device__ __forceinline__ void act_fwht_slot_xchg(float (&v)[kActSlot], float* xb, int lane) {
+#pragma unroll
+  for (int h = 1; h < kActSlot; h <<= 1) {
+#pragma unroll
+    for (int i = 0; i < kActSlot; ++i) {
+      if ((i & h) == 0) {
+        const float a = v[i];
+        const float b = v[i + h];
+        v[i] = __fadd_rn(a, b);
+        v[i + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+  const int q = lane & 7;
+  float* gb = xb + (lane >> 3) * kActXStride;
+  __syncwarp();  // earlier readers of the buffer are done
+#pragma unroll
+  for (int i = 0; i < kActSlot; ++i) gb[8 * i + 4 * (i >> 2) + q] = v[i];
+  __syncwarp();
+  // elements i = 2q (then 2q + 1), p = 0..7: 16 consecutive floats
+  const float4* r = reinterpret_cast<const float4*>(gb + 16 * q + 4 * (q >> 1));
+  float f[kActSlot];
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const float4 w = r[c];
+    f[4 * c] = w.x;
+    f[4 * c + 1] = w.y;
+    f[4 * c + 2] = w.z;
+    f[4 * c + 3] = w.w;
+  }
+  // f[8b + p] is element 16p + 2q + b
+#pragma unroll
+  for (int h = 1; h < 8; h <<= 1) {
+#pragma unroll
+    for (int p = 0; p < 8; ++p) {
+      if ((p & h) == 0) {
+#pragma unroll
+        for (int b = 0; b < 2; ++b) {
+          const float x0 = f[8 * b + p];
+          const float x1 = f[8 * b + p + h];
+          f[8 * b + p] = __fadd_rn(x0, x1);
+          f[8 * b + p + h] = __fsub_rn(x0, x1);
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    v[2 * p] = f[p];
+    v[2 * p + 1] = f[8 + p];
+  }
+}
+
+// Quantise a slot left by act_fwht_slot_xchg (t[2p + b] = element
+// 16p + 2q + b) and store the group's codes in element order: pairs of bytes
+// into the group's cb window (conflict-free: groups 36 words apart), then
+// each lane's own 16 bytes to p (when `in`).
+__device__ __forceinline__ void act_store_slot_xchg(int8_t* out, const float (&t)[kActSlot], float inv,
+                                                    uint8_t* cb, int lane, bool in) {
+  const int q = lane & 7;
+  uint8_t* gc = cb + (lane >> 3) * kActCStride;
+  __syncwarp();  // earlier readers of the buffer are done
+#pragma unroll
+  for (int p = 0; p < 8; ++p) {
+    int c0 = __float2int_rn(__fmul_rn(t[2 * p], inv));
+    int c1 = __float2int_rn(__fmul_rn(t[2 * p + 1], inv));
+    c0 = max(-127, min(127, c0));
+    c1 = max(-127, min(127, c1));
+    *reinterpret_cast<uint16_t*>(gc + 16 * p + 2 * q) =
+        static_cast<uint16_t>((static_cast<uint32_t>(c0) & 0xFFu) | ((static_cast<uint32_t>(c1) & 0xFFu) << 8));
+  }
+  __syncwarp();
+  if (in) *reinterpret_cast<uint4*>(out) = *reinterpret_cast<const uint4*>(gc + 16 * q);
+}
+
 __device__ __forceinline__ float act_slot_absmax(const float (&v)[kActSlot]) {
   float m = 0.0f;
 #pragma unroll
@@ -98,10 +187,14 @@ template <int J>
 __global__ void __launch_bounds__(kActRegMaxThreads) act_quant_reg_kernel(const uint16_t* __restrict__ x, int k, int rotate,
                                                             int8_t* __restrict__ xq, float* __restrict__ xs) {
   __shared__ float red[32];
+  // per warp: the chunk exchange of the transform and the codes' reorder
+  __shared__ __align__(16) float xbuf[kActRegMaxThreads / 32][4 * kActXStride];
+  __shared__ __align__(16) uint8_t cbuf[kActRegMaxThreads / 32][4 * kActCStride];
   pdl_launch_dependents();  // the next kernel may start its set-up
   const int64_t row = blockIdx.x;
   const int slots = k / kActSlot;
   const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   const uint16_t* xr = x + row * k;
   float v[J][kActSlot];
   float amax = 0.0f;
@@ -114,7 +207,7 @@ __global__ void __launch_bounds__(kActRegMaxThreads) act_quant_reg_kernel(const 
 #pragma unroll
       for (int i = 0; i < kActSlot; ++i) v[j][i] = 0.0f;
     }
-    if (rotate) act_fwht_slot(v[j], lane);  // whole 8-lane groups are in or out
+    if (rotate) act_fwht_slot_xchg(v[j], xbuf[warp], lane);  // whole 8-lane groups are in or out
     amax = fmaxf(amax, act_slot_absmax(v[j]));
   }
   amax = act_block_max(amax, red);
@@ -123,7 +216,11 @@ __global__ void __launch_bounds__(kActRegMaxThreads) act_quant_reg_kernel(const 
 #pragma unroll
   for (int j = 0; j < J; ++j) {
     const int s = threadIdx.x + j * blockDim.x;
-    if (s < slots) act_store_slot(qr + s * kActSlot, v[j], inv);
+    if (rotate) {
+      act_store_slot_xchg(qr + s * kActSlot, v[j], inv, cbuf[warp], lane, s < slots);
+    } else if (s < slots) {
+      act_store_slot(qr + s * kActSlot, v[j], inv);
+    }
   }
   if (threadIdx.x == 0) xs[row] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
 }
