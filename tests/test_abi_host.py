@@ -218,3 +218,57 @@ def test_pack_cb4_byte_identical_to_oracle(L):
         p, s_none, s = oracle.pack_search(w, "cb4", rotate)
         assert sub is None and s_none is None
         assert np.array_equal(codes, p) and np.array_equal(scale, s)
+
+
+def test_later_calls_reject_bad_arguments_before_any_launch(L):
+    """The codebook format, rescoring, the no-allocation linear and the
+    one-call layer validate on the host: none of these reaches the GPU."""
+    vp = ctypes.c_void_p
+    aligned = vp(1 << 20)
+    odd = vp((1 << 20) + 8)
+
+    def weight(**kw):
+        d = dict(fmt=2, rotated=1, n=256, k=512, codes=1 << 20, sub_scale=0, scale=1 << 22)
+        d.update(kw)
+        return iq8r._Weight(d["fmt"], d["rotated"], d["n"], d["k"], d["codes"], d["sub_scale"], d["scale"])
+
+    cb = weight()
+    # the codebook format runs on its GEMV only, and needs K % 128 == 0
+    assert L.iq8r_linear_ex(aligned, aligned, 4, ctypes.byref(cb), aligned, iq8r.IQ8R_PATH_TC, None) == \
+        iq8r.IQ8R_ERR_UNSUPPORTED
+    assert "GEMV only" in iq8r.iq8r_last_error()
+    assert L.iq8r_linear_ex(aligned, aligned, 4, ctypes.byref(weight(k=200)), aligned, 0, None) == \
+        iq8r.IQ8R_ERR_INVALID_ARG
+
+    trunk = weight(fmt=0, sub_scale=1 << 21)
+    cand = aligned
+
+    def rescore(w=trunk, m=8, xq=aligned, xs=aligned, c=cand, nc=32, out=aligned):
+        return L.iq8r_rescore(xq, xs, m, ctypes.byref(w), c, nc, out, None)
+
+    assert rescore(nc=-1) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert rescore(nc=65535 * 32 + 1) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert rescore(w=weight(fmt=0, sub_scale=1 << 21, k=49408)) == iq8r.IQ8R_ERR_UNSUPPORTED
+    assert rescore(w=cb) == iq8r.IQ8R_ERR_UNSUPPORTED
+    assert rescore(c=None) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert rescore(xq=odd) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert rescore(m=-1) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert rescore(m=0) == iq8r.IQ8R_OK and rescore(nc=0) == iq8r.IQ8R_OK
+
+    # the no-allocation linear checks like iq8r_linear
+    assert L.iq8r_linear_noalloc(aligned, aligned, 4, ctypes.byref(weight(fmt=0, sub_scale=0)), aligned, None) == \
+        iq8r.IQ8R_ERR_INVALID_ARG
+    assert L.iq8r_linear_noalloc(aligned, aligned, 4, ctypes.byref(trunk), odd, None) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert L.iq8r_linear_noalloc(aligned, aligned, 0, ctypes.byref(trunk), aligned, None) == iq8r.IQ8R_OK
+
+    # the one-call layer: beyond one launch it stages the codes, so it needs
+    # xq_out and x_scale_out
+    assert L.iq8r_linear_bf16(aligned, 16, ctypes.byref(trunk), aligned, None, None, None) == \
+        iq8r.IQ8R_ERR_INVALID_ARG
+    assert "xq_out" in iq8r.iq8r_last_error()
+    assert L.iq8r_linear_bf16(None, 1, ctypes.byref(trunk), aligned, None, None, None) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert L.iq8r_linear_bf16(aligned, 1, ctypes.byref(trunk), odd, None, None, None) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert L.iq8r_linear_bf16(aligned, 0, ctypes.byref(trunk), aligned, None, None, None) == iq8r.IQ8R_OK
+
+    # the self-test's limit is checked before its launch
+    assert L.iq8r_selftest_wait_timeout(10, None) == iq8r.IQ8R_ERR_INVALID_ARG
