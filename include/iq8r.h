@@ -220,9 +220,9 @@ iq8r_status iq8r_linear_noalloc(const int8_t* xq, const float* x_scale, int64_t 
 
 /* Candidate rescoring: the linear's outputs for a short list of weight rows
  * per token, out[t][j] = y[t][cand[t][j]] with y as iq8r_linear defines it
- * (same block sums, same epilogue). The IQ8R page, row "Speculator": the
- * drafter's 2-bit head proposes 32 candidates per position, which the engine
- * rescores against the model's own int8 head.
+ * (same block sums, same epilogue). The IQ8R page, row "Speculator": 32
+ * candidates a position come from the drafter's 2-bit head, and the int8
+ * head of the model itself re-scores them.
  *   xq, x_scale  as for iq8r_linear (xq 16-byte aligned)
  *   w            any IQ8R weight (the lm_head: G128); k <= 49152
  *   cand         device int32 [m][n_cand], row indices in [0, w->n)

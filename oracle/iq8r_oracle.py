@@ -79,8 +79,8 @@ __all__ = [
     "rescore",
 ]
 
-GROUP_TRUNK = 256  # trunk: one u8 scale per row and 256 of K (IQ8R page, "Weights")
-GROUP_HEAD = 128   # lm_head: one bf16 scale per row and 128 of K (IQ8R page, "Weights")
+GROUP_TRUNK = 256  # trunk: a u8 sub-scale for every (row, 256-wide block of K) (IQ8R page, "Weights")
+GROUP_HEAD = 128   # lm_head: a bf16 scale for every (row, 128-wide block of K) (IQ8R page, "Weights")
 CODE_MAX = 127     # codes in -127..127, clamp=sym (IQ8R page, "Weights" and recipe)
 SUB_MAX = 255      # largest u8 sub-scale (recipe: scale=u8)
 ROT = 128          # fwht128: the rotation acts on each 128 of K

@@ -2,9 +2,9 @@
 //
 // Trunk ("Qwen3.8-27B IQ8R + DFlash2 -- radiance container", table row
 // "Weights", and the recipe rule "codes=i8 group=256 scale=u8 scale2=bf16
-// block2=1x* transform=fwht128 clamp=sym"): int8 codes -127..127, a u8
-// sub-scale per (row, 256 of K) under a bf16 scale per row, each 128 of K
-// rotated first by the Hadamard transform without normalisation.
+// block2=1x* transform=fwht128 clamp=sym"): int8 codes -127..127; each row
+// has a bf16 scale and, below it, a u8 sub-scale for every 256 of K; every
+// 128 of K goes through the unnormalised Hadamard transform first.
 // lm_head (same row; recipe "codes=i8 group=128 scale=bf16 clamp=sym"): a
 // bf16 scale per (row, 128 of K).
 //

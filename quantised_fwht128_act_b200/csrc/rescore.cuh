@@ -1,8 +1,8 @@
 // Candidate rescoring: the outputs of the IQ8R linear for a short list of
 // weight rows per token. "Qwen3.8-27B IQ8R + DFlash2 -- radiance container",
-// table row "Speculator": the drafter's 2-bit vocabulary head proposes 32
-// candidates, which the engine rescores against the model's own (int8, bf16
-// scale per 128 of K) head. The arithmetic is the linear's exactly -- the
+// table row "Speculator": 32 candidates come from the drafter's 2-bit
+// vocabulary head, and the model's int8 head (a bf16 scale per 128 of K)
+// re-scores them. The arithmetic is the linear's exactly -- the
 // same exact int32 block sums P and the same epilogue -- evaluated only at
 // out[t][j] = y[t][cand[t][j]].
 //
