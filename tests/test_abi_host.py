@@ -272,3 +272,16 @@ def test_later_calls_reject_bad_arguments_before_any_launch(L):
 
     # the self-test's limit is checked before its launch
     assert L.iq8r_selftest_wait_timeout(10, None) == iq8r.IQ8R_ERR_INVALID_ARG
+
+
+def test_pack_accepts_torch_bf16_tensors(L):
+    """The binding takes a CPU torch bf16 tensor as well as raw bit patterns
+    and packs the same bytes."""
+    import torch
+    _, w = gen_workload("decode", m=1, n=24, k=512, seed=29)
+    t = torch.from_numpy(w.view(np.int16)).view(torch.bfloat16)
+    for fmt in ("g256", "g128", "cb4"):
+        a = iq8r.iq8r_pack(w, fmt, True)
+        b = iq8r.iq8r_pack(t, fmt, True)
+        for x, y in zip(a, b):
+            assert (x is None and y is None) or np.array_equal(x, y)
