@@ -37,10 +37,9 @@ library follows it exactly):
 
 Also written here: ``pack_search`` (the recipes' rule=search: least-error
 scales among the RTN scale and the 15 below it, for all three formats),
-``pack_cb4`` / ``decode_cb4``
-(the drafter's 16-level codebook: nearest level under s = bf16 of A / 127
-rounded up, ties to the larger level) and ``rescore`` (the layer at a list of
-candidate rows).
+``pack_cb4`` / ``decode_cb4`` (the drafter's 16-level codebook: nearest level
+under s = bf16 of A / 127 rounded up, ties to the larger level) and
+``rescore`` (the layer at a list of candidate rows).
 
 Parity unpinned: the choice of the scale rules above (per-token activation
 scale, the s2/s1 composition, the lm_head scale rule, the search window and
