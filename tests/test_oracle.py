@@ -322,3 +322,27 @@ def test_cb4_ties_and_zero_group():
     assert oracle.bf16_to_f32(scale)[0, 0] == 1.0
     assert list(v[0, :4]) == [127, -97, 6, 43]
     assert scale[1, 0] == 0 and np.all(packed[1] == 0x88)
+
+
+def test_cb4_linear_brute_force():
+    """The codebook linear against a pure-Python sum on a tiny case: every
+    index read from its nibble, looked up in the 16 levels, multiplied by the
+    token's code, summed per 128-block with integers, then scaled."""
+    table = [-127, -97, -75, -58, -43, -30, -18, -6, 6, 18, 30, 43, 58, 75, 97, 127]
+    x, w = gen_workload("decode", m=2, n=3, k=256, seed=47)
+    packed, scale = oracle.pack_cb4(w, True)
+    q, a = oracle.act_quant(x)
+    y64 = oracle.linear(q, a, "cb4", packed, None, scale, rotated=True)
+    s = oracle.bf16_to_f32(scale)
+    for m in range(2):
+        for n in range(3):
+            tot = 0.0
+            for g in range(2):
+                p = 0
+                for kk in range(g * 128, (g + 1) * 128):
+                    byte = int(packed[n, kk // 2])
+                    idx = byte & 15 if kk % 2 == 0 else byte >> 4
+                    p += int(q[m, kk]) * table[idx]
+                tot += float(s[n, g]) * p
+            want = float(np.float32(a[m])) * tot / 128.0
+            assert abs(y64[m, n] - want) <= 1e-12 * max(1.0, abs(want))

@@ -194,3 +194,18 @@ def test_rescore_of_the_neighbouring_row_is_caught(monkeypatch):
     monkeypatch.setattr(oracle, "rescore", next_row)
     with pytest.raises(AssertionError):
         test_oracle.test_rescore_is_the_linear_at_the_candidates("g256")
+
+
+def test_cb4_scale_of_the_next_block_is_caught(monkeypatch):
+    """The codebook linear scaling each block by its neighbour's scale."""
+    import test_oracle
+    real = om.linear
+
+    def shifted(xq, a, fmt, codes, sub, scale_bits, rotated=True):
+        if fmt == "cb4":
+            scale_bits = np.roll(np.asarray(scale_bits), 1, axis=1)
+        return real(xq, a, fmt, codes, sub, scale_bits, rotated)
+
+    monkeypatch.setattr(oracle, "linear", shifted)
+    with pytest.raises(AssertionError):
+        test_oracle.test_cb4_linear_brute_force()
