@@ -28,7 +28,8 @@ library follows it exactly):
 * fp32 transform order: radix-2 butterflies, h = 1, 2, 4, ..., 64, each
   (a, b) -> (a + b, a - b) with round-to-nearest-even, no fused ops;
 * activation scale: one per token (row), a = amax / 127, codes
-  rint(x' * (127 / amax)) clamped to +-127;
+  rint(x' * (127 / amax)) clamped to +-127; a row whose amax is below 2^-64
+  is first multiplied by 2^64 (exact), so that 127 / amax stays finite;
 * trunk scales: step d[n, g] = float(s2[n]) * s1[n, g]; s2 = bf16 of
   R[n] / (127 * 255) rounded up, s1 = min(255, ceil(A[n, g] / (127 * s2)));
 * lm_head scale: s[n, g] = bf16 of A[n, g] / 127 rounded up;
@@ -83,6 +84,10 @@ GROUP_HEAD = 128   # lm_head: a bf16 scale for every (row, 128-wide block of K) 
 CODE_MAX = 127     # codes in -127..127, clamp=sym (IQ8R page, "Weights" and recipe)
 SUB_MAX = 255      # largest u8 sub-scale (recipe: scale=u8)
 ROT = 128          # fwht128: the rotation acts on each 128 of K
+# Rows whose rotated absmax is below ACT_TINY are quantised after an exact
+# multiplication by ACT_PRESCALE (see act_quant).
+ACT_TINY = np.float32(2.0 ** -64)
+ACT_PRESCALE = np.float32(2.0 ** 64)
 # The drafter's 16-level integer codebook (IQ8R page, "How this file was
 # made": the dflash recipe lines, table=-127;-97;...;97;127, group=128
 # scale=bf16 transform=fwht128): index i (4 bits) stands for CB4_TABLE[i].
@@ -204,10 +209,18 @@ def act_quant(x_bits: np.ndarray, rotate: bool = True):
     "Activations"). The granularity is not given; the stated definition is per token (row):
 
       x' = fwht128(x) in float32 (or x itself when ``rotate`` is false),
-      amax = max |x'|, inv = 127 / amax (float32 divide),
-      q = clamp(rint(x' * inv), -127, 127), a = amax / 127 (float32).
+      amax = max |x'|, a = amax / 127 (float32 divide),
+      c = 2^64 if amax < 2^-64 else 1 (a power of two: x' c and amax c are exact),
+      inv = 127 / (amax c) (float32 divide),
+      q = clamp(rint((x' c) * inv), -127, 127).
 
-    A row with amax == 0 gives a = 0 and all-zero codes.
+    For every row whose 127 / amax is a finite float32 the factor c changes
+    no code: (x' c) * (127 / (amax c)) is the same real number as
+    x' * (127 / amax), so it rounds the same way. It only defines the rows
+    with amax < 127 / FLT_MAX (about 3.7e-37), where 127 / amax overflows.
+    A row with amax == 0 gives a = 0 and all-zero codes. Rows whose x' is not
+    finite (non-finite inputs, or a transform that overflows float32) are
+    outside the definition.
     Returns (q int8 [M, K], a float32 [M]).
     """
     x = bf16_to_f32(x_bits)
@@ -219,8 +232,9 @@ def act_quant(x_bits: np.ndarray, rotate: bool = True):
     a = np.zeros(xr.shape[0], dtype=np.float32)
     nz = amax > 0
     if np.any(nz):
-        inv = np.float32(CODE_MAX) / amax[nz]
-        t = xr[nz] * inv[:, None]
+        c = np.where(amax[nz] < ACT_TINY, ACT_PRESCALE, np.float32(1.0)).astype(np.float32)
+        inv = np.float32(CODE_MAX) / (amax[nz] * c)
+        t = (xr[nz] * c[:, None]) * inv[:, None]
         q[nz] = np.clip(np.rint(t), -CODE_MAX, CODE_MAX).astype(np.int8)
         a[nz] = amax[nz] / np.float32(CODE_MAX)
     return q, a

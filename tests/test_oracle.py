@@ -6,6 +6,7 @@ import torch
 
 import oracle
 import pins
+from iq8r_inputs import f32_to_bf16_bits
 from iq8r_inputs import WORKLOADS, gen_workload
 
 
@@ -76,6 +77,32 @@ def test_act_golden():
 def test_act_properties(pr1, decode_small):
     pins.check_act_properties(oracle.act_quant, oracle.fwht128_f64, pr1[0])
     pins.check_act_properties(oracle.act_quant, oracle.fwht128_f64, decode_small[0])
+
+
+def test_act_tiny_rows():
+    """Rows whose amax is below 2^-64, down to bf16 subnormals: hand-derived
+    goldens, and the general properties, with no overflow or invalid
+    operation anywhere in the oracle."""
+    pins.check_act_tiny_golden(oracle.act_quant)
+    rng = np.random.default_rng(21)
+    k = 512
+    x = rng.standard_normal((6, k))
+    x[0] *= 1e-39                                        # bf16 subnormals, amax ~ 1e-37
+    x[1] *= 2.0 ** -140                                  # mostly zeros and the smallest subnormals
+    x[2] *= 2.0 ** -70                                   # prescaled, 127 / amax finite
+    x[3] *= 2.0 ** -64                                   # around the threshold
+    x[4] = 0.0
+    x[4, 5] = 2.0 ** -133                                # a single smallest bf16 subnormal
+    x[5] *= np.exp(rng.uniform(-95, -85, k))             # mixed tiny magnitudes
+    bits = f32_to_bf16_bits(x.astype(np.float32))
+    with np.errstate(over="raise", invalid="raise", divide="raise"):
+        q, a = oracle.act_quant(bits)
+        pins.check_act_properties(oracle.act_quant, oracle.fwht128_f64, bits)
+    assert np.all(np.abs(q[a > 0]).max(axis=1) == 127)
+    # the prescale changes no code of a row whose 127 / amax is finite: the
+    # same row scaled by 2^60 (an exact bf16 exponent shift) is not prescaled
+    up = pins.bf16(pins.bf16_val(bits[2]) * np.float32(2.0 ** 60)).reshape(1, k)
+    assert np.array_equal(q[2], oracle.act_quant(up)[0][0])
 
 
 def test_act_spike_and_zero_rows():

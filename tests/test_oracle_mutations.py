@@ -209,3 +209,33 @@ def test_cb4_scale_of_the_next_block_is_caught(monkeypatch):
     monkeypatch.setattr(oracle, "linear", shifted)
     with pytest.raises(AssertionError):
         test_oracle.test_cb4_linear_brute_force()
+
+
+def test_dropped_tiny_row_prescale_is_caught(monkeypatch):
+    """Without the 2^64 factor, 127 / amax overflows for a row of bf16
+    subnormals and every code becomes +-127."""
+    monkeypatch.setattr(om, "ACT_PRESCALE", np.float32(1.0))
+    with np.errstate(over="ignore", invalid="ignore"):
+        fails(lambda: pins.check_act_tiny_golden(om.act_quant))
+
+
+def _act_prescale_variant(scale_a, scale_x):
+    """The oracle's act_quant with the 2^64 prescale misapplied."""
+    def act(x_bits, rotate=True):
+        xr = om.fwht128_f32(om.bf16_to_f32(x_bits))
+        amax = np.abs(xr).max(axis=1)
+        c = np.where(amax < om.ACT_TINY, om.ACT_PRESCALE, np.float32(1.0)).astype(np.float32)
+        inv = np.float32(127) / (amax * c)
+        t = (xr * c[:, None] if scale_x else xr) * inv[:, None]
+        q = np.clip(np.rint(t), -127, 127).astype(np.int8)
+        a = ((amax * c) if scale_a else amax) / np.float32(127)
+        return q, a.astype(np.float32)
+    return act
+
+
+def test_scale_from_the_prescaled_amax_is_caught():
+    fails(lambda: pins.check_act_tiny_golden(_act_prescale_variant(scale_a=True, scale_x=True)))
+
+
+def test_prescale_of_amax_only_is_caught():
+    fails(lambda: pins.check_act_tiny_golden(_act_prescale_variant(scale_a=False, scale_x=False)))
