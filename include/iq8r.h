@@ -25,7 +25,10 @@
  *  - the fp32 transform runs radix-2 butterflies h = 1, 2, ..., 64 in that
  *    order, (a, b) -> (a + b, a - b), round-to-nearest-even, no fused ops;
  *  - activations carry one fp32 scale per token: a = amax / 127,
- *    codes = clamp(rint(x' * (127 / amax)), -127, 127);
+ *    codes = clamp(rint(x' * (127 / amax)), -127, 127); a row with amax
+ *    below 2^-64 is first multiplied by 2^64 (exact), which keeps 127 / amax
+ *    finite down to bf16 subnormals and changes no code where it was finite;
+ *    rows whose x' is not finite are outside the definition;
  *  - trunk weights: step d[n][g] = s2[n] * s1[n][g], s2 = bf16 of
  *    R[n] / 32385 rounded up (R = row absmax of T(W)), s1 = min(255,
  *    ceil(A[n][g] / (127 * s2))) (A = absmax of the 256-block);
@@ -83,7 +86,11 @@ typedef enum {
 typedef enum {
   IQ8R_PATH_AUTO = 0,
   IQ8R_PATH_GEMV = 1,   /* weight-streaming dp4a GEMV, M handled 8 rows at a time */
-  IQ8R_PATH_TC = 2      /* tcgen05 kind::i8 tensor-core GEMM */
+  IQ8R_PATH_TC = 2,     /* tcgen05 kind::i8 tensor-core GEMM */
+  /* Flag, OR-ed into the path of iq8r_linear_ex: the weight arrays may have
+   * been written by the kernel just before this call on the stream, so read
+   * them only after that kernel has completed (see iq8r_weight). */
+  IQ8R_PATH_FLAG_WEIGHTS_WRITTEN = 0x100
 } iq8r_path;
 
 /* A packed weight on the device. Not owned by the library.
@@ -94,7 +101,17 @@ typedef enum {
  *   rotated   1 if the codes live in the fwht128 domain (the output is then
  *             multiplied by 1/128); 0 for a plain int8 weight.
  * k must be a multiple of 256 (G256) or 128 (G128); codes, sub_scale and
- * scale must be 16-byte aligned (the arrays' base addresses). */
+ * scale must be 16-byte aligned (the arrays' base addresses).
+ *
+ * Read-ahead of the weights. The linear calls launch their kernels with
+ * programmatic dependent launch: the weight-streaming kernels start copying
+ * weight tiles while the previous kernel on the stream is still finishing,
+ * and wait for it only before they read the activations. So the weight
+ * arrays must not be written by the kernel that immediately precedes a
+ * linear call on the same stream (for example a device-side repack or
+ * update): write them earlier, synchronise, or pass
+ * IQ8R_PATH_FLAG_WEIGHTS_WRITTEN to iq8r_linear_ex, which makes every kernel
+ * wait for the previous one before its first weight read. */
 typedef struct {
   int32_t fmt;
   int32_t rotated;
@@ -195,7 +212,10 @@ iq8r_status iq8r_linear(const int8_t* xq, const float* x_scale, int64_t m, const
 iq8r_status iq8r_linear_bf16(const uint16_t* x_bf16, int64_t m, const iq8r_weight* w, uint16_t* y_bf16,
                              int8_t* xq_out, float* x_scale_out, cudaStream_t stream);
 
-/* iq8r_linear with an explicit kernel choice (tests and measurement). */
+/* iq8r_linear with an explicit kernel choice (tests and measurement).
+ * path: IQ8R_PATH_AUTO, _GEMV or _TC, optionally OR IQ8R_PATH_FLAG_WEIGHTS_WRITTEN
+ * (weights written by the previous kernel on the stream; see iq8r_weight).
+ * Any other value returns IQ8R_ERR_INVALID_ARG. */
 iq8r_status iq8r_linear_ex(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w,
                            uint16_t* y_bf16, int32_t path, cudaStream_t stream);
 

@@ -22,6 +22,7 @@ import numpy as np
 __all__ = [
     "IQ8R_OK", "IQ8R_ERR_INVALID_ARG", "IQ8R_ERR_UNSUPPORTED", "IQ8R_ERR_CUDA", "IQ8R_ERR_DEVICE_TIMEOUT",
     "IQ8R_FMT_G256_U8_BF16", "IQ8R_FMT_G128_BF16", "IQ8R_PATH_AUTO", "IQ8R_PATH_GEMV", "IQ8R_PATH_TC",
+    "IQ8R_PATH_FLAG_WEIGHTS_WRITTEN",
     "IQ8R_RULE_RTN", "IQ8R_RULE_SEARCH", "IQ8R_FMT_CB4_G128",
     "IQ8RError", "IQ8RWeight", "lib", "lib_path",
     "iq8r_version", "iq8r_last_error", "iq8r_packed_sizes", "iq8r_pack", "iq8r_rotate_quant_act",
@@ -45,6 +46,8 @@ IQ8R_FMT_CB4_G128 = 2
 IQ8R_PATH_AUTO = 0
 IQ8R_PATH_GEMV = 1
 IQ8R_PATH_TC = 2
+# OR into a path: the weights were written by the previous kernel on the stream
+IQ8R_PATH_FLAG_WEIGHTS_WRITTEN = 0x100
 
 _FMT_NAMES = {"g256": IQ8R_FMT_G256_U8_BF16, "g128": IQ8R_FMT_G128_BF16, "cb4": IQ8R_FMT_CB4_G128}
 

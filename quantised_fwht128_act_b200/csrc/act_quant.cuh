@@ -1,6 +1,8 @@
 // Activation rotate + int8 quantise: the activations are int8 in the same
 // rotated domain as the weights, W8A8 ("Qwen3.8-27B IQ8R + DFlash2 --
-// radiance container", table row "Activations"), one fp32 scale per token.
+// radiance container", table row "Activations"), one fp32 scale per token:
+// a = amax / 127, codes rint(x' * (127 / amax)) clamped to +-127, a row with
+// amax below 2^-64 first multiplied by 2^64 (exact; see act_inv).
 //
 // One CTA per token row. A thread owns "slots" of 16 consecutive elements
 // (two 16-byte bf16 loads, one 16-byte int8 store). A 128-chunk is 8 slots
@@ -151,6 +153,27 @@ __device__ __forceinline__ void act_store_slot_xchg(int8_t* out, const float (&t
   if (in) *reinterpret_cast<uint4*>(out) = *reinterpret_cast<const uint4*>(gc + 16 * q);
 }
 
+// A row whose amax is below 2^-64 is quantised after an exact multiplication
+// by 2^64, so that 127 / amax stays finite down to the smallest subnormal
+// (it overflows below 127 / FLT_MAX). For every row whose 127 / amax is
+// finite this changes no code: (x' c) * (127 / (amax c)) is the same real
+// number as x' * (127 / amax). The scale a = amax / 127 is unchanged.
+constexpr float kActTiny = 0x1p-64f;
+constexpr float kActPrescale = 0x1p64f;
+
+// 127 / amax for the codes (after the prescale), 0 for a zero row.
+__device__ __forceinline__ float act_inv(float amax) {
+  return amax > 0.0f ? __fdiv_rn(127.0f, amax < kActTiny ? __fmul_rn(amax, kActPrescale) : amax) : 0.0f;
+}
+
+// The prescale of a tiny row's values (uniform across the row's threads).
+__device__ __forceinline__ void act_prescale_slot(float (&v)[kActSlot], float amax) {
+  if (amax < kActTiny) {
+#pragma unroll
+    for (int i = 0; i < kActSlot; ++i) v[i] = __fmul_rn(v[i], kActPrescale);
+  }
+}
+
 __device__ __forceinline__ float act_slot_absmax(const float (&v)[kActSlot]) {
   float m = 0.0f;
 #pragma unroll
@@ -211,11 +234,12 @@ __global__ void __launch_bounds__(kActRegMaxThreads) act_quant_reg_kernel(const 
     amax = fmaxf(amax, act_slot_absmax(v[j]));
   }
   amax = act_block_max(amax, red);
-  const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+  const float inv = act_inv(amax);
   int8_t* qr = xq + row * k;
 #pragma unroll
   for (int j = 0; j < J; ++j) {
     const int s = threadIdx.x + j * blockDim.x;
+    act_prescale_slot(v[j], amax);
     if (rotate) {
       act_store_slot_xchg(qr + s * kActSlot, v[j], inv, cbuf[warp], lane, s < slots);
     } else if (s < slots) {
@@ -275,11 +299,12 @@ __global__ void __launch_bounds__(1024) act_quant_cluster_kernel(const uint16_t*
   float g = 0.0f;
   for (uint32_t r = 0; r < gridDim.x; ++r) g = fmaxf(g, ld_shared_cluster_f32(&part_max, r));
   cluster_sync_all();  // no CTA leaves while another still reads its maximum
-  const float inv = g > 0.0f ? __fdiv_rn(127.0f, g) : 0.0f;
+  const float inv = act_inv(g);
   int8_t* qr = xq + row * k;
 #pragma unroll
   for (int j = 0; j < J; ++j) {
     const int s = s0 + threadIdx.x + j * blockDim.x;
+    act_prescale_slot(v[j], g);
     if (s < s1) act_store_slot(qr + s * kActSlot, v[j], inv);
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) xs[row] = g > 0.0f ? __fdiv_rn(g, 127.0f) : 0.0f;
@@ -311,7 +336,7 @@ __global__ void __launch_bounds__(kActTwoPassThreads) act_quant_2pass_kernel(con
     amax = fmaxf(amax, act_slot_absmax(v));
   }
   amax = act_block_max(amax, red);
-  const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+  const float inv = act_inv(amax);
   int8_t* qr = xq + row * static_cast<int64_t>(k);
   for (int j = 0; j < iters; ++j) {
     const int s = threadIdx.x + j * blockDim.x;
@@ -322,6 +347,7 @@ __global__ void __launch_bounds__(kActTwoPassThreads) act_quant_2pass_kernel(con
       for (int i = 0; i < kActSlot; ++i) v[i] = 0.0f;
     }
     if (rotate) act_fwht_slot(v, lane);
+    act_prescale_slot(v, amax);
     if (s < slots) act_store_slot(qr + static_cast<int64_t>(s) * kActSlot, v, inv);
   }
   if (threadIdx.x == 0) xs[row] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;

@@ -160,6 +160,7 @@ __global__ void __launch_bounds__(kCb4Warps * 32, 1) cb4_gemv_kernel(const Linea
     }
   }
   const bool whole = nsteps <= STEPS;
+  if (a.weights_after_wait) pdl_wait();  // the caller says that kernel wrote them
   if (whole) {
 #pragma unroll
     for (int d = 0; d < DEPTH; ++d) load(gw + d * nw, 0, ring[d], rsc[d]);

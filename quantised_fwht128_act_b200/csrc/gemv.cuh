@@ -186,8 +186,9 @@ __device__ __forceinline__ void gemv_fused_act(const LinearArgs& a, int8_t* act,
       }
       float amax = 0.0f;
       for (int w = 0; w < nwarps; ++w) amax = fmaxf(amax, red[m * 32 + w]);
-      const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+      const float inv = act_inv(amax);
       xscale[m] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
+      act_prescale_slot(v[m], amax);
       if (static_cast<int>(threadIdx.x) < slots) act_store_slot(act + m * K + threadIdx.x * kActSlot, v[m], inv);
     }
   } else {
@@ -222,7 +223,7 @@ __device__ __forceinline__ void gemv_fused_act(const LinearArgs& a, int8_t* act,
     }
     float amax = 0.0f;
     for (int w = 0; w < nwarps; ++w) amax = fmaxf(amax, red[m * 32 + w]);
-    const float inv = amax > 0.0f ? __fdiv_rn(127.0f, amax) : 0.0f;
+    const float inv = act_inv(amax);
     xscale[m] = amax > 0.0f ? __fdiv_rn(amax, 127.0f) : 0.0f;
     const uint16_t* xr = a.x + static_cast<int64_t>(m) * K;
     for (int j = 0; j < iters; ++j) {
@@ -235,6 +236,7 @@ __device__ __forceinline__ void gemv_fused_act(const LinearArgs& a, int8_t* act,
         for (int i = 0; i < kActSlot; ++i) v[i] = 0.0f;
       }
       if (a.rotated) act_fwht_slot(v, lane);
+      act_prescale_slot(v, amax);
       if (s < slots) act_store_slot(act + m * K + s * kActSlot, v, inv);
     }
   }
@@ -378,7 +380,9 @@ __global__ void __launch_bounds__(gemv_warps(MT) * 32, 1)
   };
 
   // the first stages hold only weights, which no earlier kernel writes: they
-  // stream while the previous kernel on the stream finishes
+  // stream while the previous kernel on the stream finishes (unless the
+  // caller said that kernel wrote them)
+  if (a.weights_after_wait) pdl_wait();
   for (int b = 0; b < p.depth; ++b) issue(b);
   pdl_wait();
   if (!FUSED && threadIdx.x == 0) {

@@ -77,10 +77,13 @@ iq8r::LinearArgs make_args(const int8_t* xq, const float* xs, int64_t m, const i
 
 // Choose and launch a kernel for y or partials. fixed_scratch: the
 // no-allocation variant (split-K scratch from the static array).
-iq8r_status run_linear(const iq8r::LinearArgs& a, int32_t path, const char* fn, cudaStream_t stream,
+iq8r_status run_linear(const iq8r::LinearArgs& args, int32_t path_and_flags, const char* fn, cudaStream_t stream,
                        bool fixed_scratch = false) {
+  const int32_t path = path_and_flags & ~IQ8R_PATH_FLAG_WEIGHTS_WRITTEN;
   if (path != IQ8R_PATH_AUTO && path != IQ8R_PATH_GEMV && path != IQ8R_PATH_TC)
-    return fail(IQ8R_ERR_INVALID_ARG, "%s: unknown path %d", fn, path);
+    return fail(IQ8R_ERR_INVALID_ARG, "%s: unknown path %d", fn, path_and_flags);
+  iq8r::LinearArgs a = args;
+  a.weights_after_wait = (path_and_flags & IQ8R_PATH_FLAG_WEIGHTS_WRITTEN) ? 1 : 0;
   if (a.m == 0) return ok();
   std::string why;
   if (a.fmt == IQ8R_FMT_CB4_G128) {

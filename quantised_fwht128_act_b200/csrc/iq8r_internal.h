@@ -49,6 +49,9 @@ struct LinearArgs {
   const uint16_t* x;     // [m][k] bf16, or nullptr
   int8_t* xq_out;        // [m][k] codes written back when not null
   float* xs_out;         // [m] scales written back when not null
+  // 1: the weights may come from the previous kernel on the stream; read
+  // them only after it has completed (no read-ahead under programmatic launch)
+  int weights_after_wait;
 };
 
 // Launchers (iq8r_kernels.cu). They validate nothing: the ABI layer has.

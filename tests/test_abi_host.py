@@ -157,6 +157,8 @@ def test_gpu_calls_reject_bad_arguments_before_any_launch(L):
     assert lin(weight(), y=odd) == iq8r.IQ8R_ERR_INVALID_ARG
     assert lin(weight(), xq=None) == iq8r.IQ8R_ERR_INVALID_ARG
     assert lin(weight(), path=9) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert lin(weight(), path=0x200) == iq8r.IQ8R_ERR_INVALID_ARG          # an unknown flag
+    assert lin(weight(), path=3 | iq8r.IQ8R_PATH_FLAG_WEIGHTS_WRITTEN) == iq8r.IQ8R_ERR_INVALID_ARG
     assert lin(weight(), m=0) == iq8r.IQ8R_OK
     w = weight()
     assert L.iq8r_linear_partials(aligned, 4, ctypes.byref(w), 10, 5, aligned, 0, None) == iq8r.IQ8R_ERR_INVALID_ARG

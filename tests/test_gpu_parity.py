@@ -82,18 +82,62 @@ def test_act_bit_exact_ragged_shapes(m, k):
     assert_act_exact(x, rotate=False)
 
 
-def test_act_special_rows():
-    k = 1024
-    rng = np.random.default_rng(3)
-    x = np.zeros((6, k), np.float32)
-    x[1, 700] = -3.25                                   # spike
+def special_rows(k, seed=3):
+    """Rows at the edges of the quantiser's definition: zero, a spike, large
+    magnitudes, bf16 subnormals (amax below 127 / FLT_MAX, where the 2^64
+    prescale defines the codes), small rows that are prescaled while
+    127 / amax stays finite, exact integers and mixed magnitudes."""
+    rng = np.random.default_rng(seed)
+    x = np.zeros((10, k), np.float32)
+    x[1, 700 % k] = -3.25                               # spike
     x[2] = rng.standard_normal(k) * 1e35                # large, transform stays finite
     x[3] = rng.standard_normal(k) * 1e-39               # bf16 subnormals
     x[4] = np.round(rng.standard_normal(k) * 4)         # exact small integers
     x[5] = rng.standard_normal(k) * np.exp(rng.uniform(-30, 30, k))
-    bits = f32_to_bf16_bits(x)
-    assert_act_exact(bits)
-    assert_act_exact(bits, rotate=False)
+    x[6] = rng.standard_normal(k) * 2.0 ** -70          # prescaled, 127 / amax finite
+    x[7] = rng.standard_normal(k) * 2.0 ** -140         # the smallest subnormals and zeros
+    x[8, 0], x[8, 1] = 2.0 ** -130, 2.0 ** -129         # the hand-derived tiny golden row
+    x[9] = rng.standard_normal(k) * np.exp(rng.uniform(-95, -85, k))
+    return f32_to_bf16_bits(x)
+
+
+def assert_act_exact_no_fp_traps(bits, rotate=True):
+    with np.errstate(over="raise", invalid="raise", divide="raise"):
+        assert_act_exact(bits, rotate)
+
+
+@pytest.mark.parametrize("m_rep,k", [(1, 1024), (16, 1024), (16, 17408), (1, 33024)])
+def test_act_special_rows(m_rep, k):
+    """Each activation kernel on the special rows: a cluster of CTAs a row
+    (few tokens), one CTA a row (148 tokens and up: the rows repeated), and
+    the two-pass kernel (K above 16384)."""
+    bits = np.tile(special_rows(k), (m_rep, 1))
+    assert_act_exact_no_fp_traps(bits)
+    assert_act_exact_no_fp_traps(bits, rotate=False)
+    q, a = run_act(bits)
+    # the golden row: codes 127 / -42 in the first chunk, scale 12385 * 2^-149
+    assert np.all(q[8, 0:128:2] == 127) and np.all(q[8, 1:128:2] == -42) and np.all(q[8, 128:] == 0)
+    assert a[8:9].view(np.uint32)[0] == 0x3061
+
+
+def test_act_special_rows_fused_gemv_prologue():
+    """The GEMV's fused prologue (iq8r_linear_bf16, one and two tokens)
+    writes the same codes and scales for the special rows."""
+    k, n = 1024, 64
+    bits = special_rows(k)
+    _, w = gen_workload("decode", m=1, n=n, k=k, seed=5)
+    codes, sub, scale = oracle.pack(w, "g256", True)
+    W = iq8r.IQ8RWeight.from_packed(codes, sub, scale, "g256", True)
+    with np.errstate(over="raise", invalid="raise", divide="raise"):
+        q0, a0 = oracle.act_quant(bits)
+    for i in range(0, bits.shape[0], 2):
+        xb = bits[i:i + 2]
+        xq_out = torch.empty(xb.shape, dtype=torch.int8, device="cuda")
+        xs_out = torch.empty((xb.shape[0],), dtype=torch.float32, device="cuda")
+        iq8r.iq8r_linear_bf16(dev_bf16(xb), W, xq_out=xq_out, x_scale_out=xs_out)
+        torch.cuda.synchronize()
+        assert np.array_equal(xq_out.cpu().numpy(), q0[i:i + 2])
+        assert np.array_equal(xs_out.cpu().numpy().view(np.uint32), a0[i:i + 2].view(np.uint32))
 
 
 def test_act_empty_batch_is_a_no_op():
@@ -540,3 +584,42 @@ def test_cb4_partials_window():
     vals = oracle.decode_cb4(packed)
     for n0, n1 in [(0, 5), (7, 300), (599, 600)]:
         assert np.array_equal(gpu_partials(x, W, n0, n1), oracle.partials(q, vals[n0:n1], 128))
+
+
+# ------------------------------------------------ weights written just before
+
+@pytest.mark.parametrize("fmt,path", [("g256", iq8r.IQ8R_PATH_GEMV), ("g256", iq8r.IQ8R_PATH_TC),
+                                      ("g128", iq8r.IQ8R_PATH_GEMV), ("cb4", iq8r.IQ8R_PATH_AUTO)])
+def test_weights_written_by_the_previous_kernel(fmt, path):
+    """A torch kernel rewrites the packed weight immediately before the call;
+    with IQ8R_PATH_FLAG_WEIGHTS_WRITTEN the kernels read the new weight (the
+    weight-streaming kernels otherwise read weights ahead of the previous
+    kernel's completion, see include/iq8r.h)."""
+    m, n, k = (2, 1536, 5120) if path != iq8r.IQ8R_PATH_TC else (16, 1536, 5120)
+    x, w_old = gen_workload("decode", m=m, n=n, k=k, seed=61)
+    _, w_new = gen_workload("decode", m=1, n=n, k=k, seed=62)
+    packer = (lambda w: (lambda c, s: (c, None, s))(*oracle.pack_cb4(w, True))) if fmt == "cb4" else \
+        (lambda w: oracle.pack(w, fmt, True))
+    old, new = packer(w_old), packer(w_new)
+    W = iq8r.IQ8RWeight.from_packed(*old, fmt if fmt != "cb4" else "cb4", True)
+    src = [None if a is None else torch.from_numpy(np.ascontiguousarray(a)).cuda() for a in new]
+    xq, xs = iq8r.iq8r_rotate_quant_act(dev_bf16(x))
+    torch.cuda.synchronize()
+
+    def rewrite(dst, s_):
+        if dst is None:
+            return
+        if dst.dtype == torch.uint16:
+            dst, s_ = dst.view(torch.int16), s_.view(torch.int16)
+        torch.bitwise_or(s_, 0, out=dst)  # one elementwise kernel writes dst
+
+    rewrite(W.scale, src[2])
+    rewrite(W.sub_scale, src[1])
+    rewrite(W.codes, src[0])              # the kernel right before the call
+    y = iq8r.iq8r_linear_ex(xq, xs, W, path=path | iq8r.IQ8R_PATH_FLAG_WEIGHTS_WRITTEN)
+    torch.cuda.synchronize()
+    q, a = oracle.act_quant(x)
+    y64 = oracle.linear(q, a, fmt, *new)
+    check_output(host_bits(y), y64, oracle.linear_bf16(y64))
+    iq8r.iq8r_get_device_error()
+
