@@ -212,6 +212,22 @@ iq8r_status iq8r_linear(const int8_t* xq, const float* x_scale, int64_t m, const
 iq8r_status iq8r_linear_bf16(const uint16_t* x_bf16, int64_t m, const iq8r_weight* w, uint16_t* y_bf16,
                              int8_t* xq_out, float* x_scale_out, cudaStream_t stream);
 
+/* The layer from host memory in one call: queues on `stream` the copy of
+ * x_host (bf16 [m][w->k]) into x_dev, iq8r_linear_bf16 from x_dev into
+ * y_dev, and the copy of y_dev back into y_host (bf16 [m][w->n]), and returns
+ * without waiting (synchronise the stream before reading y_host). This is
+ * the whole step of a caller whose activations live in host memory, with
+ * one crossing of the ABI instead of three.
+ *   x_host, y_host  host buffers; page-locked (cudaHostAlloc / pinned) for the
+ *                   copies to be asynchronous, else the copies are synchronous
+ *   x_dev, y_dev    caller-owned device buffers of the same sizes, 16-byte aligned
+ *   xq_out, x_scale_out  as for iq8r_linear_bf16 (needed where it needs them)
+ * Arguments are checked before the first copy is queued; a failure after
+ * that returns the failing call's status. Nothing is allocated. */
+iq8r_status iq8r_linear_bf16_host(const uint16_t* x_host, int64_t m, const iq8r_weight* w, uint16_t* x_dev,
+                                  uint16_t* y_dev, uint16_t* y_host, int8_t* xq_out, float* x_scale_out,
+                                  cudaStream_t stream);
+
 /* iq8r_linear with an explicit kernel choice (tests and measurement).
  * path: IQ8R_PATH_AUTO, _GEMV or _TC, optionally OR IQ8R_PATH_FLAG_WEIGHTS_WRITTEN
  * (weights written by the previous kernel on the stream; see iq8r_weight).

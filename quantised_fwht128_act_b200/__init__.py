@@ -26,7 +26,7 @@ __all__ = [
     "IQ8R_RULE_RTN", "IQ8R_RULE_SEARCH", "IQ8R_FMT_CB4_G128",
     "IQ8RError", "IQ8RWeight", "lib", "lib_path",
     "iq8r_version", "iq8r_last_error", "iq8r_packed_sizes", "iq8r_pack", "iq8r_rotate_quant_act",
-    "iq8r_linear", "iq8r_linear_bf16", "iq8r_linear_ex", "iq8r_linear_noalloc", "iq8r_linear_partials", "iq8r_rescore",
+    "iq8r_linear", "iq8r_linear_bf16", "iq8r_linear_bf16_host", "iq8r_linear_ex", "iq8r_linear_noalloc", "iq8r_linear_partials", "iq8r_rescore",
     "iq8r_get_device_error",
     "iq8r_selftest_wait_timeout",
 ]
@@ -103,6 +103,8 @@ def lib():
     L.iq8r_linear.argtypes = [vp, vp, i64, ctypes.POINTER(_Weight), vp, vp]
     L.iq8r_linear_bf16.restype = i32
     L.iq8r_linear_bf16.argtypes = [vp, i64, ctypes.POINTER(_Weight), vp, vp, vp, vp]
+    L.iq8r_linear_bf16_host.restype = i32
+    L.iq8r_linear_bf16_host.argtypes = [vp, i64, ctypes.POINTER(_Weight), vp, vp, vp, vp, vp, vp]
     L.iq8r_rescore.restype = i32
     L.iq8r_rescore.argtypes = [vp, vp, i64, ctypes.POINTER(_Weight), vp, i64, vp, vp]
     L.iq8r_linear_noalloc.restype = i32
@@ -219,8 +221,15 @@ class IQ8RWeight:
         return cls(f, int(bool(rotated)), c.shape[0], k, c, dev(sub), dev(scale))
 
     def _struct(self) -> _Weight:
-        return _Weight(self.fmt, self.rotated, self.n, self.k, _ptr(self.codes), _ptr(self.sub_scale),
-                       _ptr(self.scale))
+        # built once per set of buffers: a step's call then costs one
+        # comparison instead of three pointer queries and a new structure
+        key = (self.fmt, self.rotated, self.n, self.k, id(self.codes), id(self.sub_scale), id(self.scale))
+        cached = self.__dict__.get("_cached")
+        if cached is None or cached[0] != key:
+            cached = (key, _Weight(self.fmt, self.rotated, self.n, self.k, _ptr(self.codes), _ptr(self.sub_scale),
+                                   _ptr(self.scale)))
+            self.__dict__["_cached"] = cached
+        return cached[1]
 
 
 def iq8r_rotate_quant_act(x, rotate: bool = True, xq=None, x_scale=None, stream=None):
@@ -303,6 +312,19 @@ def iq8r_linear_bf16(x, weight: IQ8RWeight, y=None, xq_out=None, x_scale_out=Non
     _check(lib().iq8r_linear_bf16(_ptr(x), m, ctypes.byref(w), _ptr(y), _ptr(xq_out), _ptr(x_scale_out),
                                   _stream(stream)))
     return y
+
+
+def iq8r_linear_bf16_host(x_host, weight: IQ8RWeight, x_dev, y_dev, y_host, xq_out=None, x_scale_out=None,
+                          stream=None):
+    """One call a step from host memory: x_host (pinned bf16 [M, K]) is copied
+    to x_dev, the layer runs into y_dev, and y is copied to y_host (pinned bf16
+    [M, N]), all queued on the stream (synchronise before reading y_host).
+    xq_out / x_scale_out as for iq8r_linear_bf16 (required where the call is
+    not one launch)."""
+    m = x_host.shape[0]
+    _check(lib().iq8r_linear_bf16_host(_ptr(x_host), m, ctypes.byref(weight._struct()), _ptr(x_dev), _ptr(y_dev),
+                                       _ptr(y_host), _ptr(xq_out), _ptr(x_scale_out), _stream(stream)))
+    return y_host
 
 
 def iq8r_linear_partials(xq, weight: IQ8RWeight, n0: int = 0, n1: Optional[int] = None, p=None,

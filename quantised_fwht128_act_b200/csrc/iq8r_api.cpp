@@ -244,6 +244,29 @@ iq8r_status iq8r_linear_bf16(const uint16_t* x_bf16, int64_t m, const iq8r_weigh
   return run_linear(a, IQ8R_PATH_AUTO, fn, stream);
 }
 
+iq8r_status iq8r_linear_bf16_host(const uint16_t* x_host, int64_t m, const iq8r_weight* w, uint16_t* x_dev,
+                                  uint16_t* y_dev, uint16_t* y_host, int8_t* xq_out, float* x_scale_out,
+                                  cudaStream_t stream) {
+  const char* fn = "iq8r_linear_bf16_host";
+  iq8r_status st = check_weight(w, fn);
+  if (st != IQ8R_OK) return st;
+  if (m < 0 || m > kMaxGridRows) return fail(IQ8R_ERR_INVALID_ARG, "%s: m = %lld out of range", fn, (long long)m);
+  if (w->k % iq8r::kRot) return fail(IQ8R_ERR_INVALID_ARG, "%s: k must be a multiple of 128", fn);
+  if (m == 0) return ok();
+  if (!x_host || !y_host || !x_dev || !y_dev) return fail(IQ8R_ERR_INVALID_ARG, "%s: NULL buffer", fn);
+  if (!aligned16(x_dev) || !aligned16(y_dev) || (xq_out && !aligned16(xq_out)))
+    return fail(IQ8R_ERR_INVALID_ARG, "%s: x_dev, y_dev and xq_out must be 16-byte aligned", fn);
+  const size_t xb = static_cast<size_t>(m) * static_cast<size_t>(w->k) * 2;
+  const size_t yb = static_cast<size_t>(m) * static_cast<size_t>(w->n) * 2;
+  cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, stream);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  st = iq8r_linear_bf16(x_dev, m, w, y_dev, xq_out, x_scale_out, stream);
+  if (st != IQ8R_OK) return st;
+  e = cudaMemcpyAsync(y_host, y_dev, yb, cudaMemcpyDeviceToHost, stream);
+  if (e != cudaSuccess) return cuda_fail(e, fn);
+  return ok();
+}
+
 iq8r_status iq8r_linear(const int8_t* xq, const float* x_scale, int64_t m, const iq8r_weight* w, uint16_t* y_bf16,
                         cudaStream_t stream) {
   return iq8r_linear_ex(xq, x_scale, m, w, y_bf16, IQ8R_PATH_AUTO, stream);

@@ -272,6 +272,19 @@ def test_later_calls_reject_bad_arguments_before_any_launch(L):
     assert L.iq8r_linear_bf16(aligned, 1, ctypes.byref(trunk), odd, None, None, None) == iq8r.IQ8R_ERR_INVALID_ARG
     assert L.iq8r_linear_bf16(aligned, 0, ctypes.byref(trunk), aligned, None, None, None) == iq8r.IQ8R_OK
 
+    # the host-buffer layer checks before its first copy
+    def host(m=1, xh=aligned, xd=aligned, yd=aligned, yh=aligned, w=trunk, xq=None):
+        return L.iq8r_linear_bf16_host(xh, m, ctypes.byref(w), xd, yd, yh, xq, None, None)
+
+    assert host(xh=None) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert host(yh=None) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert host(xd=odd) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert host(yd=None) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert host(xq=odd) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert host(m=-1) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert host(w=weight(fmt=0, sub_scale=0)) == iq8r.IQ8R_ERR_INVALID_ARG
+    assert host(m=0) == iq8r.IQ8R_OK
+
     # the self-test's limit is checked before its launch
     assert L.iq8r_selftest_wait_timeout(10, None) == iq8r.IQ8R_ERR_INVALID_ARG
 

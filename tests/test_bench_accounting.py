@@ -63,3 +63,32 @@ def test_step_counts_one_launch_only_where_the_library_fuses():
     assert not bench.one_launch(1, 5120, "cb4")
     assert bench.step_bytes(8192, 5120, 17408, "g256") == \
         bench.act_bytes(8192, 5120) + bench.linear_bytes(8192, 5120, 17408, "g256")
+
+
+def test_oracle_check_reports_the_tolerance_and_bit_equality():
+    """The bench's parity summary (its CPU-baseline leg): the oracle's own
+    bf16 result passes with every output bit-equal; a result off by 2 % of
+    the RMS in one output fails the tolerance."""
+    import numpy as np
+
+    import oracle
+    from iq8r_inputs import gen_workload
+
+    x, w = gen_workload("pr1")
+    packed = oracle.pack(w, "g256", True)
+    q, a = oracle.act_quant(x)
+    y64 = oracle.linear(q, a, "g256", *packed)
+    good = oracle.linear_bf16(y64)
+    chk = {"config": "pr1", "x": x, "packed": packed, "y": good}
+    r = bench.oracle_check(chk)
+    # the literal ratio of a correctly rounded bf16 result is its own rounding
+    # (above 1e-2 of RMS here), which the half-ulp term of the reading admits
+    assert r["within_tolerance"] and r["bit_equal_frac"] == 1.0 and r["max_err_over_rms"] < 2e-2
+    rms = float(np.sqrt(np.mean(y64 ** 2)))
+    bad = oracle.linear_bf16(y64 + np.where(np.arange(y64.size).reshape(y64.shape) == 5, 0.02 * rms, 0.0))
+    r = bench.oracle_check(dict(chk, y=bad))
+    assert not r["within_tolerance"] and r["bit_equal_frac"] < 1.0
+
+
+def test_timed_reps():
+    assert bench.timed_reps(20) == 50 and bench.timed_reps(500) == 3 and bench.timed_reps(2000) == 1

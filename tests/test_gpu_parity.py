@@ -623,3 +623,29 @@ def test_weights_written_by_the_previous_kernel(fmt, path):
     check_output(host_bits(y), y64, oracle.linear_bf16(y64))
     iq8r.iq8r_get_device_error()
 
+
+# --------------------------------------------------------- host-buffer layer
+
+@pytest.mark.parametrize("name,m,n,k", [("decode", 1, 4096, 5120), ("verify16", 16, 1024, 17408)])
+def test_linear_bf16_host_matches_the_device_call(name, m, n, k):
+    """iq8r_linear_bf16_host (pinned host x in, host y out, one call) gives
+    the same bits as iq8r_linear_bf16 on device buffers, twice in a row."""
+    x, _, fmt, packed, W = case(name, m=m, n=n, k=k)
+    xd = dev_bf16(x)
+    staged = m > 2
+    xq = torch.empty(x.shape, dtype=torch.int8, device="cuda") if staged else None
+    xs = torch.empty((m,), dtype=torch.float32, device="cuda") if staged else None
+    ref = iq8r.iq8r_linear_bf16(xd, W, xq_out=xq, x_scale_out=xs)
+    xh = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).pin_memory()
+    x_dev = torch.empty_like(xd)
+    y_dev = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    for _ in range(2):
+        yh = torch.full((m, n), 7.0, dtype=torch.bfloat16).pin_memory()
+        iq8r.iq8r_linear_bf16_host(xh, W, x_dev, y_dev, yh, xq, xs)
+        torch.cuda.synchronize()
+        assert torch.equal(yh.view(torch.int16), ref.cpu().view(torch.int16))
+    q, a = oracle.act_quant(x)
+    y64 = oracle.linear(q, a, fmt, *packed)
+    check_output(yh.view(torch.int16).numpy().view(np.uint16), y64, oracle.linear_bf16(y64))
+    iq8r.iq8r_get_device_error()
+
