@@ -77,8 +77,9 @@ typedef enum {
    * even K position in the low nibble, and a bf16 scale per (row, 128 of K);
    * y as for G128 with the codes' levels. Packed by nearest level (ties to
    * the larger) under s = bf16 of A / 127 rounded up (IQ8R_RULE_RTN) or the
-   * searched scale (IQ8R_RULE_SEARCH). GEMV only (any M, 8 tokens a launch);
-   * not for iq8r_rescore. */
+   * searched scale (IQ8R_RULE_SEARCH). Weight-streaming kernels only (no
+   * IQ8R_PATH_TC): one token on dp4a, two or more on mma.sync (16 tokens a
+   * launch); not for iq8r_rescore. */
   IQ8R_FMT_CB4_G128 = 2
 } iq8r_format;
 

@@ -535,8 +535,11 @@ def linear(xq: np.ndarray, a: np.ndarray, fmt: str, codes: np.ndarray,
 
     Trunk: y = a[m] * s2[n] * S[m, n] / 128, S = sum_g s1[n, g] * P[m, n, g]
     (S exact in int64). lm_head: y = a[m] / 128 * sum_g s[n, g] * P[m, n, g]
-    (each term and the sum exact in float64). The 1/128 undoes H H = 128 I
-    and is dropped when the weight was packed unrotated.
+    in float64: each term is exact (8 significant bits of the bf16 scale
+    times an integer below 2^22), the sum of the K/128 terms is rounded, with
+    a relative error of order (K/128) 2^-53, far below any tolerance used.
+    The 1/128 undoes H H = 128 I and is dropped when the weight was packed
+    unrotated.
     """
     a64 = np.asarray(a, dtype=np.float32).astype(np.float64)
     if fmt == "g256":

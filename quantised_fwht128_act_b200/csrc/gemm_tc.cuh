@@ -78,6 +78,7 @@ struct TcParams {
   uint16_t* y;        // [m][n], or nullptr in partials mode
   int32_t* partials;  // [m][n][k/G] in partials mode
   uint32_t tmem_cols; // columns allocated: 2 * bm rounded up to a power of two >= 32
+  int weights_after_wait;  // 1: no weight tile before the previous kernel completes
 };
 
 // ------------------------------------------------------------ tcgen05 / TMA
@@ -251,10 +252,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  // set-up above overlaps the previous kernel's tail; its outputs (the
-  // activation codes and scales) are read only after it has completed
+  // set-up above overlaps the previous kernel's tail. Its outputs (the
+  // activation codes and scales) are read only after it has completed, and
+  // this kernel's own outputs are written only after that too; the producer
+  // streams the first ring of weight tiles before it waits (the weights are
+  // no earlier kernel's output, unless the caller says otherwise)
   pdl_launch_dependents();
-  pdl_wait();
+  if (warp != 0 || p.weights_after_wait) pdl_wait();
 
   // A unit is one output tile over one K range: blocks [g0, g1) of the tile's
   // ng scale blocks, split s of S (the tile's K split evenly in blocks).
@@ -271,6 +275,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       const uint64_t pol_w = p.stream_w ? l2_policy_evict_first() : l2_policy_evict_normal();
       const uint64_t pol_x = l2_policy_evict_last();
       const uint32_t tx = kTcStageA + bm * kTcStageK;
+      // the first `pre` stages' weight tiles go out before the wait for the
+      // previous kernel; their activation tiles follow it
+      uint32_t pre = 0;
+      if (!p.weights_after_wait) {
+        for (int64_t u = blockIdx.x; u < p.units && pre < static_cast<uint32_t>(nst); u += gridDim.x) {
+          int64_t tile;
+          int split, g0, g1;
+          unit_range(u, tile, split, g0, g1);
+          const int n0 = static_cast<int>((tile / p.tiles_m) * kTcBN);
+          for (int kb = g0 * SPB; kb < g1 * SPB && pre < static_cast<uint32_t>(nst); ++kb, ++pre) {
+            mbar_arrive_expect_tx(&full[pre], tx);
+            tma_load_2d(stage_base + pre * p.stage_bytes, &tmap_w, kb * kTcStageK, n0, &full[pre], pol_w);
+          }
+        }
+        pdl_wait();
+      }
       uint32_t it = 0;   // stages issued
       int st = 0;        // ring slot of stage `it`
       uint32_t ph = 0;   // its use count & 1
@@ -282,12 +302,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const int m0 = static_cast<int>((tile % p.tiles_m) * bm);
         const int n0 = static_cast<int>((tile / p.tiles_m) * kTcBN);
         for (int kb = g0 * SPB; kb < g1 * SPB; ++kb, ++it) {
+          uint8_t* sp = stage_base + st * p.stage_bytes;
+          if (it < pre) {
+            // armed and its weight tile issued before the wait
+            tma_load_2d(sp + kTcStageA, &tmap_x, kb * kTcStageK, m0, &full[st], pol_x);
+            if (++st == nst) {
+              st = 0;
+              ph ^= 1u;
+            }
+            continue;
+          }
           if (s_abort || (it >= static_cast<uint32_t>(nst) && !mbar_wait(&empty[st], ph ^ 1u, kDevErrTcEmpty))) {
             s_abort = 1;
             ok = false;
             break;
           }
-          uint8_t* sp = stage_base + st * p.stage_bytes;
           mbar_arrive_expect_tx(&full[st], tx);
           tma_load_2d(sp, &tmap_w, kb * kTcStageK, n0, &full[st], pol_w);
           tma_load_2d(sp + kTcStageA, &tmap_x, kb * kTcStageK, m0, &full[st], pol_x);
@@ -298,6 +327,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
       // never leave with a copy still landing in this CTA's shared memory
+      // (stages armed before the wait count as issued: their weight tiles are)
+      if (it < pre) it = pre;
       const uint32_t first = it > static_cast<uint32_t>(nst) ? it - nst : 0u;
       for (uint32_t j = first; j < it; ++j)
         if (!mbar_wait(&full[j % nst], (j / nst) & 1u, kDevErrTcDrain)) break;

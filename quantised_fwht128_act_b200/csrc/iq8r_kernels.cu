@@ -12,6 +12,7 @@
 #include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "cb4_gemv.cuh"
+#include "cb4_mma.cuh"
 #include "rescore.cuh"
 #include "iq8r_device.cuh"
 #include "iq8r_internal.h"
@@ -503,6 +504,7 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_
   p.scale = a.scale;
   p.y = a.y;
   p.partials = a.partials;
+  p.weights_after_wait = a.weights_after_wait;
   p.nacc = std::max(2, std::min(kTcMaxAcc, 512 / p.bm));
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(p.nacc * p.bm)) cols <<= 1;
@@ -533,6 +535,12 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_
                 : launch_tc_t<0, false, kTcMaxBM>(tw, tx, p, grid, stream);
   return part ? launch_tc_t<1, true, kTcMaxBM>(tw, tx, p, grid, stream)
               : launch_tc_t<1, false, kTcMaxBM>(tw, tx, p, grid, stream);
+}
+
+// The mma.sync codebook kernel stages 16 tokens of codes (and its
+// reduction buffer) in shared memory.
+bool cb4_mma_fits(int64_t k, const DeviceInfo& d) {
+  return 16 * (k + 16) + 4 * 32 * 4 * 2 * 4 <= d.smem_optin - kSmemReserve;
 }
 
 template <int MT, bool PARTIALS, int STEPS, bool EXACT>
@@ -570,14 +578,42 @@ cudaError_t launch_cb4_t(const LinearArgs& a, const DeviceInfo& d, cudaStream_t 
   }
 }
 
-// The codebook format: groups of up to 8 tokens a launch (their codes staged
-// in shared memory).
+template <int NT>
+cudaError_t launch_cb4_mma_t(const LinearArgs& a, const DeviceInfo& d, cudaStream_t stream) {
+  auto kernel = cb4_mma_kernel<NT>;
+  const int smem = 8 * NT * (static_cast<int>(a.k) + 16) + 4 * 32 * 4 * NT * 4;
+  static std::atomic<int> configured[kMaxDevices];
+  cudaError_t e = ensure_smem(kernel, smem, configured);
+  if (e != cudaSuccess) return e;
+  const int64_t groups = (a.n + 15) / 16;
+  const unsigned grid = static_cast<unsigned>((groups + 3) / 4);
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pdl_config(dim3(grid), dim3(kCb4MmaWarps * 32), static_cast<size_t>(smem), stream, attr);
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
+// The codebook format. Two or more tokens: mma.sync, 16 tokens a launch
+// (their codes staged in shared memory); one token, and the partial sums:
+// the dp4a kernel, up to 8 tokens a launch.
 cudaError_t launch_cb4(const LinearArgs& a, cudaStream_t stream) {
   if (a.m == 0 || a.n == 0) return cudaSuccess;
   DeviceInfo d;
   cudaError_t e = device_info(&d);
   if (e != cudaSuccess) return e;
   const int64_t ng = a.k / kGroupHead;
+  if (a.partials == nullptr && a.m >= 2 && cb4_mma_fits(a.k, d)) {
+    for (int64_t m0 = 0; m0 < a.m; m0 += 16) {
+      const int mg = static_cast<int>(std::min<int64_t>(16, a.m - m0));
+      LinearArgs s = a;
+      s.m = mg;
+      s.xq = a.xq + m0 * a.k;
+      s.xs = a.xs + m0;
+      s.y = a.y + m0 * a.n;
+      e = mg > 8 ? launch_cb4_mma_t<2>(s, d, stream) : launch_cb4_mma_t<1>(s, d, stream);
+      if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+  }
   for (int64_t m0 = 0; m0 < a.m; m0 += 8) {
     const int mg = static_cast<int>(std::min<int64_t>(8, a.m - m0));
     LinearArgs s = a;
