@@ -186,10 +186,11 @@ iq8r_status iq8r_rotate_quant_act(const uint16_t* x_bf16, int64_t m, int64_t k, 
  * Kernels: m <= 2 streams the weights through the GEMV; larger m runs the
  * tensor-core GEMM (measured on B200: from 3 tokens on it is as fast or
  * faster, at every workload shape). When the GEMM has fewer output tiles than SMs it splits
- * K: the fp32 partial tiles go to a per-device workspace (16 MiB, allocated
- * by the first such call on the device and kept for the process, so make
- * that first call before any stream capture) and a second kernel adds them
- * in a fixed order, so the result does not depend on timing. Calls on
+ * K: the fp32 partial tiles go to a per-device workspace, a 16 MiB array in
+ * the library's device image (loaded with the module; no call allocates),
+ * and a second kernel adds them in a fixed order, so the result does not
+ * depend on timing. The first call on a device looks up the array's address
+ * and sets kernel attributes: make it before any stream capture. Calls on
  * different streams that both split K and overlap in time share that
  * workspace and race; order them on one stream. Results are the same bits
  * from call to call. */
@@ -240,8 +241,8 @@ iq8r_status iq8r_linear_ex(const int8_t* xq, const float* x_scale, int64_t m, co
  * interface for callers that must not allocate, e.g. inside their own
  * memory pools or graphs). Same arguments, same kernel choice and same
  * split plan as iq8r_linear, so y is the same bits; but the split-K partial
- * tiles go to a fixed array of 8 MiB in the library's own device image
- * instead of an allocated workspace.
+ * tiles go to a fixed array of 8 MiB of its own in the library's device
+ * image (separate from iq8r_linear's workspace).
  *   - Set-up: the first call on a device looks up that array's address
  *     (cudaGetSymbolAddress) and sets kernel attributes; make it before any
  *     stream capture. No call allocates or frees device memory.

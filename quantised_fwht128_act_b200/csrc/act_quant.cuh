@@ -131,6 +131,20 @@ __device__ __forceinline__ void act_fwht_slot_xchg(float (&v)[kActSlot], float* 
   }
 }
 
+// The code of one value: rint(v * inv). No clamp is needed for a finite
+// row: |v| <= amax (after the same prescale as amax) and inv = RN(127 /
+// amax), so |v * inv| <= 127 (1 + 2^-24) and its rounding to the nearest
+// integer is at most 127 in magnitude; the clamp to +-127 of the definition
+// never acts. (Non-finite rows are outside the definition.)
+__device__ __forceinline__ int act_code(float v, float inv) { return __float2int_rn(__fmul_rn(v, inv)); }
+
+// Low bytes of four codes, in order, as one word (two byte permutes).
+__device__ __forceinline__ uint32_t act_pack4(int q0, int q1, int q2, int q3) {
+  const uint32_t lo = __byte_perm(static_cast<uint32_t>(q0), static_cast<uint32_t>(q1), 0x0040u);
+  const uint32_t hi = __byte_perm(static_cast<uint32_t>(q2), static_cast<uint32_t>(q3), 0x0040u);
+  return __byte_perm(lo, hi, 0x5410u);
+}
+
 // Quantise a slot left by act_fwht_slot_xchg (t[2p + b] = element
 // 16p + 2q + b) and store the group's codes in element order: pairs of bytes
 // into the group's cb window (conflict-free: groups 36 words apart), then
@@ -142,12 +156,10 @@ __device__ __forceinline__ void act_store_slot_xchg(int8_t* out, const float (&t
   __syncwarp();  // earlier readers of the buffer are done
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
-    int c0 = __float2int_rn(__fmul_rn(t[2 * p], inv));
-    int c1 = __float2int_rn(__fmul_rn(t[2 * p + 1], inv));
-    c0 = max(-127, min(127, c0));
-    c1 = max(-127, min(127, c1));
+    const int c0 = act_code(t[2 * p], inv);  // in -127..127 (see act_code)
+    const int c1 = act_code(t[2 * p + 1], inv);
     *reinterpret_cast<uint16_t*>(gc + 16 * p + 2 * q) =
-        static_cast<uint16_t>((static_cast<uint32_t>(c0) & 0xFFu) | ((static_cast<uint32_t>(c1) & 0xFFu) << 8));
+        static_cast<uint16_t>(__byte_perm(static_cast<uint32_t>(c0), static_cast<uint32_t>(c1), 0x0040u));
   }
   __syncwarp();
   if (in) *reinterpret_cast<uint4*>(out) = *reinterpret_cast<const uint4*>(gc + 16 * q);
@@ -182,13 +194,11 @@ __device__ __forceinline__ float act_slot_absmax(const float (&v)[kActSlot]) {
 }
 
 __device__ __forceinline__ void act_store_slot(int8_t* p, const float (&v)[kActSlot], float inv) {
-  uint32_t w[4] = {0u, 0u, 0u, 0u};
+  uint32_t w[4];
 #pragma unroll
-  for (int i = 0; i < kActSlot; ++i) {
-    int q = __float2int_rn(__fmul_rn(v[i], inv));
-    q = max(-127, min(127, q));
-    w[i >> 2] |= (static_cast<uint32_t>(q) & 0xFFu) << (8 * (i & 3));
-  }
+  for (int i = 0; i < 4; ++i)
+    w[i] = act_pack4(act_code(v[4 * i], inv), act_code(v[4 * i + 1], inv), act_code(v[4 * i + 2], inv),
+                     act_code(v[4 * i + 3], inv));
   *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 

@@ -118,6 +118,30 @@ __device__ __forceinline__ void bulk_g2s_default(void* dst, const void* src, uin
                : "memory");
 }
 
+// Plan the copy of bytes [o0, o1) of a 16-byte-aligned array of `total`
+// bytes into dst as the 16-byte-aligned window [o0 & ~15, ...) around them,
+// one bulk copy; dst[(o0 & 15) + i] is then byte o0 + i. Only bytes past the
+// last whole 16 of the array (the final rows of a matrix) go by plain loads,
+// done here (by the lane with copy_tail) before the caller's arrive.
+struct GemvWindow {
+  const uint8_t* src;
+  uint8_t* dst;
+  uint32_t bytes;
+};
+__device__ __forceinline__ GemvWindow window_copy_plan(uint8_t* dst, const uint8_t* base, int64_t total, int64_t o0,
+                                                       int64_t o1, bool copy_tail) {
+  const int64_t w0 = o0 & ~int64_t(15);
+  const int64_t e16 = total & ~int64_t(15);
+  int64_t w1 = (o1 + 15) & ~int64_t(15);
+  if (w1 > e16) {
+    w1 = e16;
+    if (copy_tail)
+      for (int64_t b = (w0 > e16 ? w0 : e16); b < o1; ++b) dst[b - w0] = __ldg(base + b);
+  }
+  GemvWindow w{base + w0, dst, w1 > w0 ? static_cast<uint32_t>(w1 - w0) : 0u};
+  return w;
+}
+
 // Named barrier over `threads` threads (a multiple of 32), id 1..15.
 __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");

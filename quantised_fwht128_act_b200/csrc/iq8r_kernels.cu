@@ -3,7 +3,6 @@
 
 #include <algorithm>
 #include <atomic>
-#include <mutex>
 #include <string>
 
 #include <cudaTypedefs.h>
@@ -334,23 +333,26 @@ cudaError_t make_tmap_i8(CUtensorMap* map, const void* base, int64_t rows, int64
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-// Split-K workspace, one per device, made on the first split launch there:
-// the fp32 partial tiles of the units.
+// Split-K workspace: the fp32 partial tiles of the units, in an array of the
+// library's device image (made when the module is loaded on a device, kept
+// for the process), so no call allocates. Its address is looked up once per
+// device.
 constexpr size_t kTcWsBytes = size_t(16) << 20;
+static __device__ __align__(256) float g_tc_ws_array[kTcWsBytes / sizeof(float)];
 float* g_tc_ws[kMaxDevices];
-std::mutex g_tc_ws_mu;
+std::atomic<int> g_tc_ws_ready[kMaxDevices];
 
 cudaError_t tc_workspace(float** out) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> lock(g_tc_ws_mu);
-  if (g_tc_ws[dev] == nullptr) {
-    void* a = nullptr;
-    e = cudaMalloc(&a, kTcWsBytes);
+  if (g_tc_ws_ready[dev].load(std::memory_order_acquire) == 0) {
+    void* ptr = nullptr;
+    e = cudaGetSymbolAddress(&ptr, g_tc_ws_array);
     if (e != cudaSuccess) return e;
-    g_tc_ws[dev] = static_cast<float*>(a);
+    g_tc_ws[dev] = static_cast<float*>(ptr);
+    g_tc_ws_ready[dev].store(1, std::memory_order_release);
   }
   *out = g_tc_ws[dev];
   return cudaSuccess;
