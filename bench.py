@@ -349,37 +349,42 @@ def run_ours(args, rank, world, local_rank):
     stream.synchronize()
     iq8r.iq8r_get_device_error(stream)
 
-    # graphs: a main chunk of C steps (a multiple of R) and a tail. A step of
-    # one launch is captured bare, so consecutive launches keep their
-    # programmatic (overlapping) dependency and the kernel's average launch is
-    # the timed region / K; a step of two kernels is bracketed by external
-    # events so the graph records each kernel's timestamps.
+    # graphs: a main chunk of C steps (a multiple of R) and a tail, captured
+    # bare, so consecutive kernels keep their programmatic (overlapping)
+    # dependency, as a caller's stream would: the timed region replays these.
+    # A step of two kernels is also captured once with external events
+    # around each kernel (an event between two kernels removes their
+    # overlap), replayed outside the timed region for the per-kernel times.
     C = min(K, max(R, (512 // R) * R))
     n_main, tail = divmod(K, C)
 
-    def capture(nsteps, offset):
+    def capture(nsteps, offset, with_events=False):
         try:
             g = torch.cuda.CUDAGraph(keep_graph=True)  # kept so its kernel nodes can be counted
         except TypeError:
             g = torch.cuda.CUDAGraph()
-        evs = None if fused else [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
-                                  for _ in range(nsteps)]
+        evs = None if not with_events else [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+                                            for _ in range(nsteps)]
         with torch.cuda.graph(g, stream=stream):
             for j in range(nsteps):
                 r = (offset + j) % R
                 if fused:
                     iq8r.iq8r_linear_bf16(x_dev[r], weights[r], y[r])
                     continue
-                evs[j][0].record()
+                if with_events:
+                    evs[j][0].record()
                 iq8r.iq8r_rotate_quant_act(x_dev[r], True, xq[r], xsc[r])
-                evs[j][1].record()
+                if with_events:
+                    evs[j][1].record()
                 linear(r)
-                evs[j][2].record()
+                if with_events:
+                    evs[j][2].record()
         g.instantiate()
         return g, evs
 
-    g_main, ev_main = capture(C, 0) if n_main else (None, None)
-    g_tail, ev_tail = capture(tail, 0) if tail else (None, None)
+    g_main, _ = capture(C, 0) if n_main else (None, None)
+    g_tail, _ = capture(tail, 0) if tail else (None, None)
+    g_ev, evs_ev = (None, None) if fused else capture(min(K, C), 0, with_events=True)
     # this library's kernel launches inside the timed region: the kernel
     # nodes of each captured graph times its replays
     counts = [graph_kernel_nodes(g) for g in (g_main, g_tail)]
@@ -431,10 +436,6 @@ def run_ours(args, rank, world, local_rank):
         regions.append(max_over_ranks(start.elapsed_time(end), world, dev))
         if fused:
             lin_ms.append(regions[-1] / K)
-        else:
-            evs = ev_main if ev_main is not None else ev_tail
-            act_ms.append(float(np.mean([e[0].elapsed_time(e[1]) for e in evs])))
-            lin_ms.append(float(np.mean([e[1].elapsed_time(e[2]) for e in evs])))
     t_end_wall = time.time()
     if world > 1:
         torch.distributed.barrier()
@@ -443,8 +444,16 @@ def run_ours(args, rank, world, local_rank):
     iq8r.iq8r_get_device_error(stream)
     if fused:
         act_ms = [0.0]
+    else:
+        # per-kernel durations, each kernel on its own (outside the timed region)
+        for _ in range(3):
+            with torch.cuda.stream(stream):
+                g_ev.replay()
+            stream.synchronize()
+            act_ms.append(float(np.mean([e[0].elapsed_time(e[1]) for e in evs_ev])))
+            lin_ms.append(float(np.mean([e[1].elapsed_time(e[2]) for e in evs_ev])))
     elapsed_ms = float(np.median(regions))
-    del g_main, g_tail
+    del g_main, g_tail, g_ev
 
     # end to end through the public API: every step is one call of
     # iq8r_linear_bf16_host, which queues the pinned H2D copy of x, the layer
@@ -558,7 +567,9 @@ def run_ours(args, rank, world, local_rank):
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
                    "timing": (("CUDA graphs of the K launches (programmatic dependent launch); events around "
                                "the timed region, average launch = region / K") if fused else
-                              "CUDA graphs of the K steps; events inside the graphs time each kernel")
+                              ("CUDA graphs of the K steps, kernels back to back (programmatic dependent launch); "
+                               "per-kernel times from a copy of the graph with events around each kernel, "
+                               "replayed outside the timed region"))
                              + f"; the K-step region timed {reps} times back to back, median reported"},
         "roofline": roof,
         "clocks": clocks,

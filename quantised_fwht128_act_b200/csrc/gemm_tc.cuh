@@ -550,57 +550,4 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
 }
 
-// Split-K second pass: y[m][n] = bf16(sum over splits, in split order, of
-// the fp32 partial tiles, times a[m] * s2[n] / 128 (trunk) or a[m] / 128
-// (lm_head)). One thread: one weight row of one tile, 8 consecutive tokens;
-// consecutive threads take consecutive rows, so output stores coalesce.
-constexpr int kTcReduceThreads = 256;
-template <int FMT>
-__global__ void __launch_bounds__(kTcReduceThreads) tc_split_reduce_kernel(const TcParams p) {
-  pdl_wait();  // the partial tiles come from the kernel before
-  const int chunks = p.bm / 8;
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= p.tiles * kTcBN * chunks) return;
-  const int64_t tile = i / (kTcBN * chunks);
-  const int rem = static_cast<int>(i - tile * kTcBN * chunks);
-  const int r = rem % kTcBN;
-  const int ch = rem / kTcBN;
-  const int64_t m0 = (tile % p.tiles_m) * p.bm + ch * 8;
-  const int64_t n = (tile / p.tiles_m) * kTcBN + r;
-  if (n >= p.n || m0 >= p.m) return;
-  const size_t sstride = static_cast<size_t>(kTcBN) * p.bm;
-  const float* w = p.ws + static_cast<size_t>(tile) * p.splits * sstride + static_cast<size_t>(r) * p.bm + ch * 8;
-  float acc[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
-  for (int sp0 = 0; sp0 < p.splits; sp0 += 4) {
-    float4 v[4][2];
-#pragma unroll
-    for (int t = 0; t < 4; ++t)
-      if (sp0 + t < p.splits) {
-        const float4* q = reinterpret_cast<const float4*>(w + (sp0 + t) * sstride);
-        v[t][0] = __ldcg(q);
-        v[t][1] = __ldcg(q + 1);
-      }
-#pragma unroll
-    for (int t = 0; t < 4; ++t)
-      if (sp0 + t < p.splits) {
-        acc[0] += v[t][0].x;
-        acc[1] += v[t][0].y;
-        acc[2] += v[t][0].z;
-        acc[3] += v[t][0].w;
-        acc[4] += v[t][1].x;
-        acc[5] += v[t][1].y;
-        acc[6] += v[t][1].z;
-        acc[7] += v[t][1].w;
-      }
-  }
-  const float rs = (FMT == 0 ? bf16_bits_to_float(p.scale[n]) : 1.0f) * (p.rotated ? 0.0078125f : 1.0f);
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int64_t m = m0 + j;
-    if (m < p.m) __stcs(p.y + m * p.n + n, float_to_bf16_bits_rn(acc[j] * p.xs[m] * rs));
-  }
-}
-
 }  // namespace iq8r

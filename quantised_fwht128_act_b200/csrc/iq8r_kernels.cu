@@ -9,6 +9,7 @@
 
 #include "act_quant.cuh"
 #include "gemm_tc.cuh"
+#include "tc_split_reduce.cuh"
 #include "gemv.cuh"
 #include "cb4_gemv.cuh"
 #include "cb4_mma.cuh"
@@ -426,7 +427,7 @@ cudaError_t launch_tc_t(const CUtensorMap& tw, const CUtensorMap& tx, const TcPa
   cudaLaunchConfig_t cfg = pdl_config(dim3(grid), dim3(kTcThreads), kTcSmemBytes, stream, attr);
   e = cudaLaunchKernelEx(&cfg, kernel, tw, tx, p);
   if (e != cudaSuccess || p.splits <= 1) return e;
-  const int64_t threads = p.tiles * kTcBN * (p.bm / 8);
+  const int64_t threads = p.tiles * kTcBN * (p.bm / 4);
   cudaLaunchConfig_t rcfg = pdl_config(dim3(static_cast<unsigned>((threads + kTcReduceThreads - 1) / kTcReduceThreads)),
                                        dim3(kTcReduceThreads), 0, stream, attr);
   return cudaLaunchKernelEx(&rcfg, tc_split_reduce_kernel<FMT>, p);
