@@ -531,13 +531,15 @@ def run_ours(args, rank, world, local_rank):
         # the burst figure for a short timed region, the sustained one when the
         # clock record shows the power cap during it
         achieved_t = ops / (lin_avg_ms * 1e-3) / 1e12
-        capped = "sw_power_cap" in (sampler.summary(t_start_wall, t_end_wall).get("reasons") or [])
+        ck = sampler.summary(t_start_wall, t_end_wall)
+        capped = ("sw_power_cap" in (ck.get("reasons") or []) and ck.get("sm_mhz") is not None
+                  and ck.get("sm_max_mhz") is not None and ck["sm_mhz"] < ck["sm_max_mhz"])
         bf16_use = sustained_bf16() if capped else bf16_tf
         peak_i8 = bf16_use * INT8_OVER_BF16
         roof = {"bound": "tensor", "kernel": kname, "achieved": achieved_t,
                 "peak": peak_i8, "unit": "TOPS", "frac": achieved_t / peak_i8,
                 "peak_source": (f"{peak_src} cuBLAS bf16 {bf16_use:.1f} TFLOP/s (MEASURED_PEAKS.json "
-                                f"{'bf16_tflops_sustained: the power cap was active' if capped else 'bf16_tflops'}) "
+                                f"{'bf16_tflops_sustained: the power cap held the median clock below its maximum' if capped else 'bf16_tflops'}) "
                                 f"x {INT8_OVER_BF16:g} (nominal dense int8/bf16)"),
                 "frac_of_datasheet_4500": achieved_t / 4500.0,
                 "hbm_gbs": lin_b / (lin_avg_ms * 1e-3) / 1e9,

@@ -53,6 +53,15 @@ constexpr int kTcRingBytes = kTcStages * kTcStageBytes;     // 192 KB for the op
 // ring, then barriers (2 x 12 + 2 x 8 + 1) x 8 B, the TMEM address and flags, 2 x 256
 // activation scales; plus 1 KB to align the ring to 1024 bytes
 constexpr int kTcSmemBytes = kTcRingBytes + 4096 + 1024;
+// Small token tiles (BM <= 64: verify blocks and few-token lm_head calls):
+// two CTAs an SM, each with half the operand ring and at most 256 TMEM
+// columns, so one CTA's stalls (unit boundaries, the epilogue) are covered
+// by the other's weight stream. Measured on B200 at BM = 32: verify8/16
+// 36 -> 27 us a GEMM, lm_head M = 8 213 -> 143 us.
+constexpr int kTcRingBytesSmall = 96 * 1024;
+__host__ __device__ constexpr int tc_ctas_per_sm(int bmax) { return bmax <= 64 ? 2 : 1; }
+__host__ __device__ constexpr int tc_ring_bytes(int bmax) { return bmax <= 64 ? kTcRingBytesSmall : kTcRingBytes; }
+__host__ __device__ constexpr int tc_smem_bytes(int bmax) { return tc_ring_bytes(bmax) + 4096 + 1024; }
 // Split-K partial tiles: fp32 [BM][128] per unit, BM <= 128 when split.
 constexpr int kTcSplitMaxBM = 128;
 
@@ -200,7 +209,7 @@ __device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
 // BMAX: the largest token tile the instance handles (256, or 128 for the
 // split-K capable instance, whose epilogue keeps half the registers).
 template <int FMT, bool PARTIALS, int BMAX>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, tc_ctas_per_sm(BMAX))
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmap_w, const __grid_constant__ CUtensorMap tmap_x,
                    const TcParams p) {
   constexpr int kCols = BMAX / kTcGroups;  // most tokens per epilogue column group
@@ -211,7 +220,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   // 1024-byte alignment for the swizzled TMA tiles
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* stage_base = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kTcRingBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + tc_ring_bytes(BMAX));
   uint64_t* empty = full + kTcMaxStages;
   uint64_t* acc_full = empty + kTcMaxStages;
   uint64_t* acc_empty = acc_full + kTcMaxAcc;

@@ -420,11 +420,12 @@ template <int FMT, bool PARTIALS, int BMAX>
 cudaError_t launch_tc_t(const CUtensorMap& tw, const CUtensorMap& tx, const TcParams& p, int grid,
                         cudaStream_t stream) {
   auto kernel = gemm_tc_kernel<FMT, PARTIALS, BMAX>;
+  constexpr int smem = tc_smem_bytes(BMAX);
   static std::atomic<int> configured[kMaxDevices];
-  cudaError_t e = ensure_smem(kernel, kTcSmemBytes, configured);
+  cudaError_t e = ensure_smem(kernel, smem, configured);
   if (e != cudaSuccess) return e;
   cudaLaunchAttribute attr[1];
-  cudaLaunchConfig_t cfg = pdl_config(dim3(grid), dim3(kTcThreads), kTcSmemBytes, stream, attr);
+  cudaLaunchConfig_t cfg = pdl_config(dim3(grid), dim3(kTcThreads), smem, stream, attr);
   e = cudaLaunchKernelEx(&cfg, kernel, tw, tx, p);
   if (e != cudaSuccess || p.splits <= 1) return e;
   const int64_t threads = p.tiles * kTcBN * (p.bm / 4);
@@ -470,16 +471,18 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_
   p.tiles_m = (a.m + p.bm - 1) / p.bm;
   p.tiles = p.tiles_m * ((a.n + kTcBN - 1) / kTcBN);
   p.stage_bytes = kTcStageA + p.bm * kTcStageK;
-  p.stages = std::min(kTcMaxStages, kTcRingBytes / p.stage_bytes);
+  const int bmax = p.bm <= 32 ? 32 : (p.bm <= 64 ? 64 : (p.bm <= kTcSplitMaxBM ? kTcSplitMaxBM : kTcMaxBM));
+  const int slots = d.num_sms * tc_ctas_per_sm(bmax);
+  p.stages = std::min(kTcMaxStages, tc_ring_bytes(bmax) / p.stage_bytes);
   p.stream_w = p.tiles_m == 1 ? 1 : 0;
   // split K when there are too few tiles to fill the SMs
   const int ng = static_cast<int>(a.k / (a.fmt == 0 ? kGroupTrunk : kGroupHead));
   p.splits = 1;
   if (p.bm <= kTcSplitMaxBM && a.partials == nullptr) {
-    double best = tc_split_cost(p.tiles, ng, 1, d.num_sms);
+    double best = tc_split_cost(p.tiles, ng, 1, slots);
     for (int S = 2; S <= std::min(ng, 32); ++S) {
       if (static_cast<size_t>(p.tiles) * S * p.bm * kTcBN * sizeof(float) > kTcWsBytes) break;
-      const double c = tc_split_cost(p.tiles, ng, S, d.num_sms);
+      const double c = tc_split_cost(p.tiles, ng, S, slots);
       if (c < 0.95 * best) {
         best = c;
         p.splits = S;
@@ -508,7 +511,8 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_
   p.y = a.y;
   p.partials = a.partials;
   p.weights_after_wait = a.weights_after_wait;
-  p.nacc = std::max(2, std::min(kTcMaxAcc, 512 / p.bm));
+  // accumulators: the 512 TMEM columns shared by the CTAs resident on an SM
+  p.nacc = std::max(2, std::min(kTcMaxAcc, 512 / (p.bm * tc_ctas_per_sm(bmax))));
   uint32_t cols = 32;
   while (cols < static_cast<uint32_t>(p.nacc * p.bm)) cols <<= 1;
   p.tmem_cols = cols;
@@ -517,7 +521,7 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_
   if (e != cudaSuccess) return e;
   e = make_tmap_i8(&tx, a.xq, a.m, a.k, p.bm);
   if (e != cudaSuccess) return e;
-  const int grid = static_cast<int>(std::min<int64_t>(d.num_sms, p.units));
+  const int grid = static_cast<int>(std::min<int64_t>(slots, p.units));
   const bool part = a.partials != nullptr;
   if (p.bm <= 32) {
     if (a.fmt == 0)
@@ -525,6 +529,13 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_
                   : launch_tc_t<0, false, 32>(tw, tx, p, grid, stream);
     return part ? launch_tc_t<1, true, 32>(tw, tx, p, grid, stream)
                 : launch_tc_t<1, false, 32>(tw, tx, p, grid, stream);
+  }
+  if (p.bm <= 64) {
+    if (a.fmt == 0)
+      return part ? launch_tc_t<0, true, 64>(tw, tx, p, grid, stream)
+                  : launch_tc_t<0, false, 64>(tw, tx, p, grid, stream);
+    return part ? launch_tc_t<1, true, 64>(tw, tx, p, grid, stream)
+                : launch_tc_t<1, false, 64>(tw, tx, p, grid, stream);
   }
   if (p.bm <= kTcSplitMaxBM) {
     if (a.fmt == 0)
