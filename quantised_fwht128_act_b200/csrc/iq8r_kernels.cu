@@ -11,6 +11,7 @@
 #include "gemm_tc.cuh"
 #include "tc_split_reduce.cuh"
 #include "gemv.cuh"
+#include "gemv_reg.cuh"
 #include "cb4_gemv.cuh"
 #include "cb4_mma.cuh"
 #include "rescore.cuh"
@@ -131,8 +132,62 @@ cudaError_t launch_gemv_t(const LinearArgs& a, const GemvPlan& plan, const Devic
   return cudaLaunchKernelEx(&cfg, kernel, a, p, tiles / grid, tiles % grid);
 }
 
+// The register-streaming GEMV's shape (one or two tokens): rows_base == 0
+// when its activation codes and scale window do not fit shared memory.
+RegPlan gemv_reg_plan(const LinearArgs& a, int mt, const DeviceInfo& d) {
+  RegPlan p{};
+  if (mt > 2 || a.n < 1) return p;
+  const int64_t ng = a.k / (a.fmt == 0 ? kGroupTrunk : kGroupHead);
+  const int64_t grid = std::min<int64_t>(d.num_sms, a.n);
+  const int64_t rmax = (a.n + grid - 1) / grid;
+  const int64_t sc = a.fmt == 0 ? gemv_align16(static_cast<int>(std::min<int64_t>(rmax * ng, 1 << 24)) + 32) +
+                                      gemv_align16(static_cast<int>(std::min<int64_t>(2 * rmax, 1 << 24)) + 32)
+                                : gemv_align16(static_cast<int>(std::min<int64_t>(2 * rmax * ng, 1 << 24)) + 32);
+  const int64_t smem = gemv_align128(static_cast<int>(mt * a.k)) + sc;
+  if (rmax * ng > (1 << 22) || smem > d.smem_optin - kSmemReserve) return p;
+  p.rows_base = a.n / grid;
+  p.rows_extra = a.n % grid;
+  p.parts = static_cast<int>((a.k + kRegPartBytes - 1) / kRegPartBytes);
+  p.sc_bytes = static_cast<int>(sc);
+  p.smem = static_cast<int>(smem);
+  return p;
+}
+
+template <int MT, int FMT, bool FUSED, bool AFTER>
+cudaError_t launch_gemv_reg_t(const LinearArgs& a, const RegPlan& p, const DeviceInfo& d, cudaStream_t stream) {
+  auto kernel = gemv_reg_kernel<MT, FMT, FUSED, AFTER>;
+  static std::atomic<int> configured[kMaxDevices];
+  cudaError_t e = ensure_smem(kernel, p.smem, configured);
+  if (e != cudaSuccess) return e;
+  // programmatic dependent launch: the first units of weights stream while
+  // the stream's previous kernel drains (the kernel waits for it before
+  // touching activations or outputs)
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(d.num_sms, a.n)));
+  cfg.blockDim = dim3(kRegWarps * 32);
+  cfg.dynamicSmemBytes = static_cast<size_t>(p.smem);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, a, p);
+}
+
 template <int FMT, int MODE>
 cudaError_t launch_gemv_mt(const LinearArgs& a, int mt, const DeviceInfo& d, cudaStream_t stream) {
+  if (MODE != kGemvPartials) {
+    const RegPlan rp = gemv_reg_plan(a, mt, d);
+    if (rp.parts > 0) {
+      constexpr bool fused = MODE == kGemvFused;
+      if (a.weights_after_wait)
+        return mt == 1 ? launch_gemv_reg_t<1, FMT, fused, true>(a, rp, d, stream)
+                       : launch_gemv_reg_t<2, FMT, fused, true>(a, rp, d, stream);
+      return mt == 1 ? launch_gemv_reg_t<1, FMT, fused, false>(a, rp, d, stream)
+                     : launch_gemv_reg_t<2, FMT, fused, false>(a, rp, d, stream);
+    }
+  }
   const GemvPlan p = gemv_choose(mt, FMT, static_cast<int>(a.k), d);
   if (p.rt == 0) return cudaErrorInvalidConfiguration;
   // rows computed together: up to 1, 2 or 4 by token count, never past a tile

@@ -222,9 +222,12 @@ def test_linear_within_tolerance_workloads(name):
 
 
 @pytest.mark.parametrize("path", ["gemv", "auto"])
-# (1, 300, 17408) and (2, 150, 8192): rows longer than a stage, streamed in chunks
+# (1, 300, 17408) and (2, 150, 8192): rows longer than a stage, streamed in chunks;
+# (2, 7437, 2560) and (1, 7104, 4864): 48 rows a CTA or more, the last ones in
+# 1 KB parts (4864: a part of 768 bytes and a half 512-byte step)
 @pytest.mark.parametrize("m,n,k", [(1, 1000, 768), (3, 37, 2304), (13, 64, 512), (5, 9, 4352), (2, 333, 1280),
-                                   (8, 77, 1536), (1, 300, 17408), (2, 150, 8192)])
+                                   (8, 77, 1536), (1, 300, 17408), (2, 150, 8192), (2, 7437, 2560),
+                                   (1, 7104, 4864)])
 def test_linear_within_tolerance_ragged(m, n, k, path):
     x, _, fmt, packed, W = case("decode", m=m, n=n, k=k, seed=11 + m + n + k)
     y64 = oracle_linear(x, fmt, packed)
@@ -328,7 +331,8 @@ def test_bounded_wait_reports_timeout_and_context_survives():
 @pytest.mark.parametrize("name,m,n,k", [("pr1", None, None, None), ("decode", None, None, None),
                                         ("verify8", None, None, None), ("decode", 3, 1000, 768),
                                         ("decode", 5, 37, 2304), ("decode", 7, 40, 17408),
-                                        ("decode", 1, 300, 17408), ("decode", 2, 100, 8192)])
+                                        ("decode", 1, 300, 17408), ("decode", 2, 100, 8192),
+                                        ("decode", 2, 7437, 2560), ("decode", 1, 7104, 4864)])
 def test_linear_bf16_fused_matches_two_call_path(name, m, n, k):
     """One-launch act + GEMV: codes and scales bit-exact against the oracle,
     y bit-identical to the two-call path and within tolerance of the oracle."""
@@ -621,6 +625,24 @@ def test_weights_written_by_the_previous_kernel(fmt, path):
     q, a = oracle.act_quant(x)
     y64 = oracle.linear(q, a, fmt, *new)
     check_output(host_bits(y), y64, oracle.linear_bf16(y64))
+    iq8r.iq8r_get_device_error()
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 17408, 5120), (2, 7437, 2560)])
+def test_gemv_back_to_back_launches_agree(m, n, k):
+    """Five launches queued back to back on one stream (each may start while
+    the previous one drains) give the same bits as one launch alone; any
+    per-launch state of the kernel must be back in place for the next one."""
+    x, _, fmt, packed, W = case("decode", m=m, n=n, k=k, seed=71 + m)
+    xd = dev_bf16(x)
+    ref = iq8r.iq8r_linear_bf16(xd, W)
+    torch.cuda.synchronize()
+    ys = [iq8r.iq8r_linear_bf16(xd, W) for _ in range(5)]
+    xq, xs = iq8r.iq8r_rotate_quant_act(xd)
+    ys += [iq8r.iq8r_linear(xq, xs, W) for _ in range(3)]
+    torch.cuda.synchronize()
+    for y in ys:
+        assert torch.equal(y.view(torch.int16), ref.view(torch.int16))
     iq8r.iq8r_get_device_error()
 
 
