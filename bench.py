@@ -510,11 +510,15 @@ def run_ours(args, rank, world, local_rank):
     hbm_bound = is_hbm_bound(m, k, n, fmt, fused)
     on_tc = args.path == "tc" or (args.path == "auto" and not fused and m > GEMV_MAX_M)
     on_tc = on_tc and fmt != "cb4"  # the codebook format has its own GEMV only
+    # one or two tokens stream through the register-load GEMV, more (when
+    # forced onto the GEMV) through the shared-memory-stage one
+    reg = m <= 2
     kname = ("cb4_gemv_kernel" if fmt == "cb4" else
-             "gemv_kernel (fused act, one launch per step)" if fused else
-             "gemm_tc_kernel (tcgen05 kind::i8)" if on_tc else "gemv_kernel")
+             "gemm_tc_kernel (tcgen05 kind::i8)" if on_tc else
+             ("gemv_reg_kernel" if reg else "gemv_kernel") + (" (fused act, one launch per step)" if fused else ""))
     kfiles = (["cb4_gemv.cuh", "iq8r_device.cuh"] if fmt == "cb4" else
-              ["gemm_tc.cuh", "iq8r_device.cuh"] if on_tc else ["gemv.cuh", "act_quant.cuh", "iq8r_device.cuh"])
+              ["gemm_tc.cuh", "iq8r_device.cuh"] if on_tc else
+              (["gemv_reg.cuh"] if reg else []) + ["gemv.cuh", "act_quant.cuh", "iq8r_device.cuh"])
     ktraffic = recorded_traffic(kname.split(" ")[0], args.config, kfiles)
     if hbm_bound:
         achieved = lin_b / (lin_avg_ms * 1e-3) / 1e9
@@ -541,6 +545,9 @@ def run_ours(args, rank, world, local_rank):
                 "peak_source": (f"{peak_src} cuBLAS bf16 {bf16_use:.1f} TFLOP/s (MEASURED_PEAKS.json "
                                 f"{'bf16_tflops_sustained: the power cap held the median clock below its maximum' if capped else 'bf16_tflops'}) "
                                 f"x {INT8_OVER_BF16:g} (nominal dense int8/bf16)"),
+                # both measured denominators, whichever the line's frac uses
+                "frac_of_burst": achieved_t / (bf16_tf * INT8_OVER_BF16),
+                "frac_of_sustained": achieved_t / (sustained_bf16() * INT8_OVER_BF16),
                 "frac_of_datasheet_4500": achieved_t / 4500.0,
                 "hbm_gbs": lin_b / (lin_avg_ms * 1e-3) / 1e9,
                 "traffic": ktraffic,

@@ -183,7 +183,9 @@ iq8r_status iq8r_rotate_quant_act(const uint16_t* x_bf16, int64_t m, int64_t k, 
  * of K); /128 only when w->rotated. The sum over g is carried in fp32 or
  * exact integers, so y matches the float64 value to within its bf16
  * rounding plus ~1e-6 of the output's scale.
- * Kernels: m <= 2 streams the weights through the GEMV; larger m runs the
+ * Kernels: m <= 2 streams the weights through the GEMV (16-byte loads into
+ * registers, three half rows in flight a warp, the rows' block scales in
+ * shared memory); larger m runs the
  * tensor-core GEMM (measured on B200: from 3 tokens on it is as fast or
  * faster, at every workload shape). When the GEMM has fewer output tiles than SMs it splits
  * K: the fp32 partial tiles go to a per-device workspace, a 16 MiB array in
