@@ -154,20 +154,18 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) gemv_reg_kernel(const Linea
   int4 buf[NB][PS];
   int brow[NB] = {};
   int bpart[NB] = {};
-  // A unit wholly inside the row (every unit when K is a multiple of 2560)
-  // loads without per-lane guards: an inline-assembly load cannot be
-  // predicated, so a guard on each would be a branch on each.
+  // Loads carry no per-lane guard (an inline-assembly load cannot be
+  // predicated, so a guard on each would be a branch on each): a step past
+  // the row's end reads the row's last 16 bytes instead, and its weights are
+  // zeroed where they are used.
   auto load = [&](int j) {
     if (brow[j] < 0) return;
-    const int8_t* src = a.codes + (r0 + brow[j]) * K + bpart[j] * kRegPartBytes + lane * 16;
-    if ((bpart[j] + 1) * kRegPartBytes <= K) {
+    const int8_t* src = a.codes + (r0 + brow[j]) * K;
+    const int k0 = bpart[j] * kRegPartBytes + lane * 16;
 #pragma unroll
-      for (int u = 0; u < PS; ++u) buf[j][u] = AFTER ? ldg_weights_coherent(src + u * 512) : ldg_weights(src + u * 512);
-    } else {
-      const int left = K - bpart[j] * kRegPartBytes - lane * 16;  // bytes of the row from this lane's first
-#pragma unroll
-      for (int u = 0; u < PS; ++u)
-        if (u * 512 < left) buf[j][u] = AFTER ? ldg_weights_coherent(src + u * 512) : ldg_weights(src + u * 512);
+    for (int u = 0; u < PS; ++u) {
+      const int kk = min(k0 + u * 512, K - 16);
+      buf[j][u] = AFTER ? ldg_weights_coherent(src + kk) : ldg_weights(src + kk);
     }
   };
 
@@ -231,8 +229,10 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) gemv_reg_kernel(const Linea
         }
       }
       auto step = [&](int u) {
-        const int kk = (part * PS + u) * 512 + lane * 16;
-        const int4 wv = buf[j][u];
+        const int kr = (part * PS + u) * 512 + lane * 16;
+        const bool in = kr < K;  // past the row's end: zero weights (the products are 0)
+        const int kk = in ? kr : K - 16;
+        const int4 wv = in ? buf[j][u] : make_int4(0, 0, 0, 0);
         if (FMT == 0) {
           const int s1 = s1w[row * ng + kk / G];
 #pragma unroll
@@ -246,14 +246,8 @@ __global__ void __launch_bounds__(kRegWarps * 32, 1) gemv_reg_kernel(const Linea
                 fmaf(static_cast<float>(dot16(wv, *reinterpret_cast<const int4*>(act + m * K + kk))), s, facc[m]);
         }
       };
-      if ((part + 1) * kRegPartBytes <= K) {
 #pragma unroll
-        for (int u = 0; u < PS; ++u) step(u);
-      } else {
-#pragma unroll
-        for (int u = 0; u < PS; ++u)
-          if ((part * PS + u) * 512 + lane * 16 < K) step(u);
-      }
+      for (int u = 0; u < PS; ++u) step(u);
       // the registers are free again: the warp's next unit streams into them
       next_unit(brow[j], bpart[j]);
       load(j);
