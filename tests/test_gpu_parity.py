@@ -628,6 +628,32 @@ def test_weights_written_by_the_previous_kernel(fmt, path):
     iq8r.iq8r_get_device_error()
 
 
+@pytest.mark.parametrize("m,n,k", [(1, 17408, 5120), (2, 7437, 2560), (1, 300, 17408), (2, 150, 8192)])
+def test_gemv_trunk_outputs_from_exact_block_sums(m, n, k):
+    """The one- and two-token GEMV's bf16 outputs, bit for bit, rebuilt from
+    the oracle's exact block sums: S[m, n] = sum_g s1[n, g] * P[m, n, g] as an
+    exact integer, then the kernel's stated epilogue as plain IEEE float32
+    steps, ((float(S) * a[m]) * s2[n]) * (1/128), each rounded to nearest,
+    and one bf16 rounding to nearest. A dropped or repeated block, a sub-scale
+    from the wrong block or another token's codes change S and so the bits.
+    Both entries: the codes given, and the fused one."""
+    x, _, fmt, (codes, sub, scale), W = case("decode", m=m, n=n, k=k, seed=61 + m + n)
+    q, a = oracle.act_quant(x)
+    P = oracle.partials(q, codes, 256).astype(np.int64)  # [m, n, k / 256]
+    S = np.einsum("mng,ng->mn", P, sub.astype(np.int64))
+    s2 = (scale.astype(np.uint32) << 16).view(np.float32)
+    yf = S.astype(np.float32) * a.astype(np.float32)[:, None]
+    yf = (yf * s2[None, :]).astype(np.float32)
+    yf = (yf * np.float32(0.0078125)).astype(np.float32)
+    expect = oracle.bf16_round_nearest(yf.astype(np.float64))
+    xd = dev_bf16(x)
+    y_fused = host_bits(iq8r.iq8r_linear_bf16(xd, W))
+    xq, xs = iq8r.iq8r_rotate_quant_act(xd)
+    y_codes = host_bits(iq8r.iq8r_linear_ex(xq, xs, W, path=iq8r.IQ8R_PATH_GEMV))
+    assert np.array_equal(y_codes, expect), f"{np.sum(y_codes != expect)} of {expect.size} outputs differ"
+    assert np.array_equal(y_fused, expect), f"{np.sum(y_fused != expect)} of {expect.size} outputs differ"
+
+
 @pytest.mark.parametrize("m,n,k", [(1, 17408, 5120), (2, 7437, 2560)])
 def test_gemv_back_to_back_launches_agree(m, n, k):
     """Five launches queued back to back on one stream (each may start while
