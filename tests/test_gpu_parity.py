@@ -654,6 +654,71 @@ def test_gemv_trunk_outputs_from_exact_block_sums(m, n, k):
     assert np.array_equal(y_fused, expect), f"{np.sum(y_fused != expect)} of {expect.size} outputs differ"
 
 
+def _fma32(p64: np.ndarray, acc32: np.ndarray) -> np.ndarray:
+    """float32 of p + acc rounded once to nearest-even (a float32 fused
+    multiply-add whose product p is exact in float64). The sum is taken
+    exactly as s + err (two-sum); s rounds to float32 correctly unless s
+    lies on a float32 midpoint, where the sign of err decides."""
+    b = acc32.astype(np.float64)
+    s = p64 + b
+    bb = s - p64
+    err = (p64 - (s - bb)) + (b - bb)
+    r = s.astype(np.float32)
+    r64 = r.astype(np.float64)
+    lo = np.nextafter(r, np.float32(-np.inf))
+    hi = np.nextafter(r, np.float32(np.inf))
+    r = np.where((s == (r64 + hi.astype(np.float64)) / 2) & (err > 0), hi, r)
+    r = np.where((s == (r64 + lo.astype(np.float64)) / 2) & (err < 0), lo, r)
+    return r.astype(np.float32)
+
+
+def _g128_gemv_steps(xq, a, codes, scale_bits):
+    """The one- and two-token GEMV's stated lm_head arithmetic in float32 from
+    exact integer dot products: lane L of a row's warp takes 16 bytes of K a
+    512-byte step (K positions 512 s + 16 L ..; a step past K adds a zero
+    product with the last block's scale), accumulates fma(q, s_block, acc)
+    over the steps in K order, the 32 lane sums meet in a 16-8-4-2-1
+    exchange of float32 adds, and y = bf16(acc * a * (1/128))."""
+    m_tok, k = xq.shape
+    s32 = (scale_bits.astype(np.uint32) << 16).view(np.float32)
+    lanes = np.arange(32)
+    out = []
+    for m in range(m_tok):
+        acc = np.zeros((codes.shape[0], 32), dtype=np.float32)
+        for st in range(-(-k // 2560) * 5):
+            kr = st * 512 + lanes * 16
+            valid = kr < k
+            kk = np.where(valid, kr, k - 16)
+            idx = kk[:, None] + np.arange(16)[None, :]
+            q = (codes[:, idx].astype(np.int64) * xq[m, idx].astype(np.int64)[None]).sum(-1)
+            q = np.where(valid[None, :], q, 0)
+            acc = _fma32(q.astype(np.float64) * s32[:, kk // 128].astype(np.float64), acc)
+        for off in (16, 8, 4, 2, 1):
+            acc = (acc + acc[:, lanes ^ off]).astype(np.float32)
+        y = (acc[:, 0] * np.float32(a[m])).astype(np.float32)
+        out.append((y * np.float32(0.0078125)).astype(np.float32))
+    return oracle.bf16_round_nearest(np.stack(out).astype(np.float64))
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 4096, 5120), (2, 700, 1024), (1, 300, 4352)])
+def test_gemv_g128_outputs_from_exact_dot_products(m, n, k):
+    """The same for the lm_head (G128) format, whose sum over blocks is
+    float32: the GEMV's outputs bit-equal to its stated summation order over
+    the oracle's codes and exact 16-byte dot products. A scale taken from a
+    neighbouring block (it changes 4059 of the 4096 outputs at the first
+    shape), or a step dropped or summed twice, changes bits. (K = 1024 and
+    4352: a row's last unit partly past its end.)"""
+    x, _, fmt, (codes, sub, scale), W = case("lm_head8", m=m, n=n, k=k, seed=67 + m + n)
+    q, a = oracle.act_quant(x)
+    expect = _g128_gemv_steps(q, a, codes, scale)
+    xd = dev_bf16(x)
+    y_fused = host_bits(iq8r.iq8r_linear_bf16(xd, W))
+    xq, xs = iq8r.iq8r_rotate_quant_act(xd)
+    y_codes = host_bits(iq8r.iq8r_linear_ex(xq, xs, W, path=iq8r.IQ8R_PATH_GEMV))
+    assert np.array_equal(y_codes, expect), f"{np.sum(y_codes != expect)} of {expect.size} outputs differ"
+    assert np.array_equal(y_fused, expect), f"{np.sum(y_fused != expect)} of {expect.size} outputs differ"
+
+
 @pytest.mark.parametrize("m,n,k", [(1, 17408, 5120), (2, 7437, 2560)])
 def test_gemv_back_to_back_launches_agree(m, n, k):
     """Five launches queued back to back on one stream (each may start while
