@@ -226,6 +226,16 @@ iq8r_status iq8r_linear_bf16(const uint16_t* x_bf16, int64_t m, const iq8r_weigh
  *                   copies to be asynchronous, else the copies are synchronous
  *   x_dev, y_dev    caller-owned device buffers of the same sizes, 16-byte aligned
  *   xq_out, x_scale_out  as for iq8r_linear_bf16 (needed where it needs them)
+ * When x is at most 64 KB and y at most 1 MB (a decode step), both host
+ * buffers are page-locked, mapped into the current device's address space
+ * (every page-locked allocation is, under unified addressing) and 16-byte
+ * aligned, the two copies are small kernels that read x_host and write
+ * y_host through the mapping, chained with the layer by programmatic
+ * dependent launch, so back-to-back calls overlap as device-only calls do;
+ * x_host is read before the previous kernel on the stream has finished (the
+ * caller has filled it before the call). Otherwise they are copy calls (the
+ * copy engines move large buffers faster than the device's reads of host
+ * memory do).
  * Arguments are checked before the first copy is queued; a failure after
  * that returns the failing call's status. Nothing is allocated. */
 iq8r_status iq8r_linear_bf16_host(const uint16_t* x_host, int64_t m, const iq8r_weight* w, uint16_t* x_dev,

@@ -244,6 +244,22 @@ iq8r_status iq8r_linear_bf16(const uint16_t* x_bf16, int64_t m, const iq8r_weigh
   return run_linear(a, IQ8R_PATH_AUTO, fn, stream);
 }
 
+// Largest copies the host-buffer entry makes as mapped-copy kernels.
+constexpr size_t kMappedInMaxBytes = 64 * 1024;
+constexpr size_t kMappedOutMaxBytes = 1024 * 1024;
+
+// The device address of pinned host memory mapped into the current device's
+// address space, or nullptr (pageable or device memory, or an unknown
+// pointer). The query's own error state is cleared.
+static void* mapped_host(const void* p) {
+  cudaPointerAttributes at{};
+  if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return nullptr;
+  }
+  return at.type == cudaMemoryTypeHost ? at.devicePointer : nullptr;
+}
+
 iq8r_status iq8r_linear_bf16_host(const uint16_t* x_host, int64_t m, const iq8r_weight* w, uint16_t* x_dev,
                                   uint16_t* y_dev, uint16_t* y_host, int8_t* xq_out, float* x_scale_out,
                                   cudaStream_t stream) {
@@ -258,6 +274,25 @@ iq8r_status iq8r_linear_bf16_host(const uint16_t* x_host, int64_t m, const iq8r_
     return fail(IQ8R_ERR_INVALID_ARG, "%s: x_dev, y_dev and xq_out must be 16-byte aligned", fn);
   const size_t xb = static_cast<size_t>(m) * static_cast<size_t>(w->k) * 2;
   const size_t yb = static_cast<size_t>(m) * static_cast<size_t>(w->n) * 2;
+  // Small copies between pinned host buffers that the device can address
+  // run as kernels chained with the layer (see mapped_copy.cuh): there a
+  // step's cost is latency, which the chaining hides. Large inputs, or
+  // anything else (pageable memory, an unaligned view): copy calls. (On
+  // B200 a 557 KB input read through the mapping ran at about 5 GB/s, where
+  // the copy engines stream it; reads of host memory by the device are
+  // round trips, writes are not.)
+  const bool small = xb <= kMappedInMaxBytes && yb <= kMappedOutMaxBytes;
+  const uint16_t* xm = small ? static_cast<const uint16_t*>(mapped_host(x_host)) : nullptr;
+  uint16_t* ym = small ? static_cast<uint16_t*>(mapped_host(y_host)) : nullptr;
+  if (xm && ym && aligned16(xm) && aligned16(ym)) {
+    cudaError_t e = iq8r::launch_mapped_copy(xm, x_dev, m * w->k, true, stream);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    st = iq8r_linear_bf16(x_dev, m, w, y_dev, xq_out, x_scale_out, stream);
+    if (st != IQ8R_OK) return st;
+    e = iq8r::launch_mapped_copy(y_dev, ym, m * w->n, false, stream);
+    if (e != cudaSuccess) return cuda_fail(e, fn);
+    return ok();
+  }
   cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xb, cudaMemcpyHostToDevice, stream);
   if (e != cudaSuccess) return cuda_fail(e, fn);
   st = iq8r_linear_bf16(x_dev, m, w, y_dev, xq_out, x_scale_out, stream);

@@ -65,6 +65,11 @@ cudaError_t launch_gemm_tc(const LinearArgs& a, cudaStream_t stream, bool fixed_
                            bool* too_big = nullptr);
 bool gemm_tc_supported(const LinearArgs& a, std::string* why);
 cudaError_t read_and_clear_device_error(uint32_t* err);
+// n bf16 values from src to dst by a kernel (programmatic launch), one of
+// them pinned host memory mapped into the device's address space (its
+// device address), both 16-byte aligned (mapped_copy.cuh).
+cudaError_t launch_mapped_copy(const uint16_t* src, uint16_t* dst, int64_t n, bool host_to_device,
+                               cudaStream_t stream);
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream);
 // The drafter's codebook format (cb4_gemv.cuh): y or partials.
 cudaError_t launch_cb4(const LinearArgs& a, cudaStream_t stream);

@@ -12,6 +12,7 @@
 #include "tc_split_reduce.cuh"
 #include "gemv.cuh"
 #include "gemv_reg.cuh"
+#include "mapped_copy.cuh"
 #include "cb4_gemv.cuh"
 #include "cb4_mma.cuh"
 #include "rescore.cuh"
@@ -762,6 +763,22 @@ __global__ void wait_selftest_kernel(uint64_t limit_cycles) {
 }
 
 }  // namespace
+
+cudaError_t launch_mapped_copy(const uint16_t* src, uint16_t* dst, int64_t n, bool host_to_device,
+                               cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  DeviceInfo d;
+  cudaError_t e = device_info(&d);
+  if (e != cudaSuccess) return e;
+  // enough CTAs that an input copy is read ahead of the wait in one piece
+  // per thread-slot (at most kMapCopyAhead x 16 bytes a thread), at most one an SM
+  const int64_t per_cta = static_cast<int64_t>(kMapCopyThreads) * kMapCopyAhead * 8;
+  const int64_t grid = std::max<int64_t>(1, std::min<int64_t>(d.num_sms, (n + per_cta - 1) / per_cta));
+  cudaLaunchAttribute attr[1];
+  cudaLaunchConfig_t cfg = pdl_config(dim3(static_cast<unsigned>(grid)), dim3(kMapCopyThreads), 0, stream, attr);
+  return host_to_device ? cudaLaunchKernelEx(&cfg, mapped_copy_kernel<true>, src, dst, n)
+                        : cudaLaunchKernelEx(&cfg, mapped_copy_kernel<false>, src, dst, n);
+}
 
 cudaError_t launch_wait_selftest(uint64_t limit_ns, cudaStream_t stream) {
   // cycles at no more than 2 GHz: the wait lasts at most about limit_ns

@@ -741,8 +741,10 @@ def test_gemv_back_to_back_launches_agree(m, n, k):
 
 @pytest.mark.parametrize("name,m,n,k", [("decode", 1, 4096, 5120), ("verify16", 16, 1024, 17408)])
 def test_linear_bf16_host_matches_the_device_call(name, m, n, k):
-    """iq8r_linear_bf16_host (pinned host x in, host y out, one call) gives
-    the same bits as iq8r_linear_bf16 on device buffers, twice in a row."""
+    """iq8r_linear_bf16_host (pinned host x in, host y out, one call: the
+    mapped-copy kernels) gives the same bits as iq8r_linear_bf16 on device
+    buffers, twice in a row; so do pageable buffers (the copy calls) and an
+    output whose size is not a multiple of 8 values (the copy's tail)."""
     x, _, fmt, packed, W = case(name, m=m, n=n, k=k)
     xd = dev_bf16(x)
     staged = m > 2
@@ -760,5 +762,21 @@ def test_linear_bf16_host_matches_the_device_call(name, m, n, k):
     q, a = oracle.act_quant(x)
     y64 = oracle.linear(q, a, fmt, *packed)
     check_output(yh.view(torch.int16).numpy().view(np.uint16), y64, oracle.linear_bf16(y64))
+    # pageable host buffers take the copy calls instead of the mapped-copy kernels
+    xp = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16).clone()
+    yp = torch.full((m, n), 7.0, dtype=torch.bfloat16)
+    assert not xp.is_pinned() and not yp.is_pinned()
+    iq8r.iq8r_linear_bf16_host(xp, W, x_dev, y_dev, yp, xq, xs)
+    torch.cuda.synchronize()
+    assert torch.equal(yp.view(torch.int16), ref.cpu().view(torch.int16))
+    # a ragged output (m * n not a multiple of 8: the copy's element tail)
+    if m == 1:
+        Wr = iq8r.IQ8RWeight.from_packed(*[np.ascontiguousarray(t[:n - 3]) for t in packed], fmt, True)
+        ref_r = iq8r.iq8r_linear_bf16(xd, Wr)
+        yr = torch.full((m, n - 3), 7.0, dtype=torch.bfloat16).pin_memory()
+        yr_dev = torch.empty((m, n - 3), dtype=torch.bfloat16, device="cuda")
+        iq8r.iq8r_linear_bf16_host(xh, Wr, x_dev, yr_dev, yr)
+        torch.cuda.synchronize()
+        assert torch.equal(yr.view(torch.int16), ref_r.cpu().view(torch.int16))
     iq8r.iq8r_get_device_error()
 
