@@ -1,4 +1,9 @@
-// Weight-streaming IQ8R GEMV for small M (decode and short verify blocks).
+// Weight-streaming IQ8R GEMV for small M, streaming through shared-memory
+// stages filled by bulk copies. The library runs it for the partial sums
+// (the debug twin below), for a GEMV forced at three to eight tokens, and
+// where the register-streaming kernel (gemv_reg.cuh, the one- and two-token
+// path) does not fit; its fused activation prologue (gemv_fused_act) and
+// dot16 serve both.
 //
 // y[m][n] = a[m] * s2[n] * sum_g s1[n][g] * P[m][n][g] / 128 (trunk) or
 // a[m] / 128 * sum_g s[n][g] * P[m][n][g] (lm_head), P the exact int32 dot
@@ -12,8 +17,9 @@
 //  - persistent grid, one CTA per SM, each CTA a contiguous range of tiles
 //    (balanced to one tile). A tile is RT whole weight rows (contiguous in
 //    memory), or, when a row is longer than a stage, one row in K chunks;
-//  - no producer warp: each of the 8 warps owns D private stage buffers and
-//    keeps them full itself. One lane claims the next tile from a per-CTA
+//  - no producer warp: each warp (16 a CTA for one or two tokens, else 8)
+//    owns D private stage buffers and keeps them full itself. One lane
+//    claims the next tile from a per-CTA
 //    counter and issues 1-D bulk copies (TMA engine) of the stage's codes and
 //    scales (u8 sub-scales + bf16 row scales, or the lm_head's bf16 group
 //    scales) completing on the buffer's mbarrier, weights evict-first in L2.
